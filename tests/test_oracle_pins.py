@@ -1,0 +1,304 @@
+"""Pins of the CPU oracle to what the LiquidGEMM review page and plain
+mathematics fix (no GPU).
+
+Each test checks the oracle against something other than itself: the page's
+dequantization identity and overflow claim (exhaustively), the s_u8 <= 16
+bound, hand-derived group cases, error bounds that follow from the
+definitions, symmetry and scaling invariants, brute-force integer matmuls on
+tiny inputs, numpy's int64 / float64 matmul, and IEEE bf16 rounding checked
+against torch where the value is exact in fp32.
+"""
+import itertools
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _pairs():
+    return [(mn, mx) for mn in range(-119, 120) for mx in range(mn, 120)]
+
+
+def _groups_covering_every_q(pairs):
+    """Groups of 64 INT8 weights whose min is mn and max is mx and that
+    together contain every q in [mn, mx] for each (mn, mx) pair."""
+    rows, meta = [], []
+    for mn, mx in pairs:
+        qs = list(range(mn, mx + 1))
+        for i in range(0, len(qs), 62):
+            chunk = qs[i:i + 62]
+            g = [mn, mx] + chunk + [mn] * (62 - len(chunk))
+            rows.append(g)
+            meta.append((mn, mx))
+    return np.array(rows, dtype=np.int8), np.array(meta, dtype=np.int32)
+
+
+@pytest.mark.parametrize("rule", [oracle.RULE_CEIL, oracle.RULE_ROUND])
+def test_dequant_identity_and_overflow_exhaustive(rule):
+    """Review key_machinery + referee summary: for every admissible group
+    (min, max in the protective range [-119, 119], referee major 3 / Sec. 4
+    Eq. 7) and every weight in it, the UINT8 intermediate q_u4*s_u8 + a stays
+    in [0, 255], XOR 0x80 of it equals the signed value q_u4*s_u8 + min, and
+    the codes/scales stay in UINT4 / [1, 16]."""
+    pairs = _pairs()
+    assert len(pairs) == 28680
+    Q, meta = _groups_covering_every_q(pairs)
+    codes, s, a = oracle.quantize_weights_u4(Q, group=64, rule=rule)
+    s = s[:, 0].astype(np.int32)
+    a = a[:, 0].astype(np.int32)
+    mn, mx = meta[:, 0], meta[:, 1]
+    assert np.all(a == 128 + mn)                      # a = 2^7 + min(Q_i8)
+    assert s.min() >= 1 and s.max() == 16             # s_u8 <= 16, reached
+    assert codes.max() <= 15                          # UINT4 codes
+    c = codes.astype(np.int32)
+    u8 = c * s[:, None] + a[:, None]
+    assert u8.min() >= 0 and u8.max() <= 255          # never leaves UINT8
+    xor_val = ((u8 ^ 0x80) & 0xFF).astype(np.uint8).view(np.int8).astype(np.int32)
+    plain = oracle.dequant_weights(codes, s[:, None].astype(np.uint8),
+                                   a[:, None].astype(np.uint8)).astype(np.int32)
+    assert np.array_equal(xor_val, plain)             # identity holds
+    assert plain.min() >= -119 and plain.max() <= 127
+    # rounding error: ceil rule is round-to-nearest, so |err| <= s/2
+    err = np.abs(plain - Q.astype(np.int32))
+    if rule == oracle.RULE_CEIL:
+        assert np.all(2 * err <= s[:, None])
+    # scalar entry points agree with the array ones on the extreme pair
+    assert oracle.group_scale(-119, 119, rule) == 16
+    assert oracle.dequant_xor(15, 16, 9) == (121, 249)
+
+
+def test_packed_four_lane_multiply_add_has_no_carry():
+    """The kernel dequantizes four codes per 32-bit word with one integer
+    multiply-add (review key_machinery: IMAD + XOR per four elements).  For
+    every reachable (s, a) and every reachable code in each lane, the packed
+    word w*s + a*0x01010101 must equal the four lane results, i.e. no carry
+    crosses a byte."""
+    rng = np.random.default_rng(0)
+    pairs = _pairs()
+    for mn, mx in pairs[::7]:
+        s = oracle.group_scale(mn, mx)
+        a = oracle.group_offset(mn)
+        cmax = oracle.group_code(mx, mn, s)
+        lanes = rng.integers(0, cmax + 1, size=(16, 4))
+        lanes[0] = cmax
+        lanes[1] = 0
+        w = (lanes[:, 0] | lanes[:, 1] << 8 | lanes[:, 2] << 16 | lanes[:, 3] << 24)
+        packed = ((w.astype(np.uint64) * s + a * 0x01010101) & 0xFFFFFFFF) ^ 0x80808080
+        for j in range(4):
+            byte = ((packed >> (8 * j)) & 0xFF).astype(np.uint8).view(np.int8)
+            expect = [oracle.dequant_signed(c, s, a) for c in lanes[:, j]]
+            assert list(byte.astype(int)) == expect
+
+
+def test_unreachable_triples_would_overflow():
+    """The UINT8 bound depends on the quantizer: a code/scale/offset triple
+    that the quantizer never emits does leave UINT8 (so the sweep above is
+    a real check, not a tautology)."""
+    v, u8 = oracle.dequant_xor(15, 16, 247)   # mn = 119 with s = 16: unreachable
+    assert u8 > 255
+    assert oracle.group_scale(119, 119) == 1
+
+
+def _load_group_cases():
+    rows = []
+    with open(os.path.join(HERE, "golden", "lqq_group_cases.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            p = line.split()
+            rows.append((p[0],) + tuple(int(x) for x in p[1:]))
+    return rows
+
+
+@pytest.mark.parametrize("case", _load_group_cases())
+def test_hand_derived_group_cases(case):
+    rule_name, mn, mx, q, s, a, code, u8, deq = case
+    rule = oracle.RULE_CEIL if rule_name == "ceil" else oracle.RULE_ROUND
+    assert oracle.group_scale(mn, mx, rule) == s
+    assert oracle.group_offset(mn) == a
+    assert oracle.group_code(q, mn, s, rule) == code
+    v, u = oracle.dequant_xor(code, s, a)
+    assert (v, u) == (deq, u8)
+    assert oracle.dequant_signed(code, s, a) == deq
+    # the same case through the array quantizer on a real group
+    g = np.array([[mn, mx, q] + [mn] * 61], dtype=np.int8)
+    c, ss, aa = oracle.quantize_weights_u4(g, 64, rule)
+    assert (int(ss[0, 0]), int(aa[0, 0]), int(c[0, 2])) == (s, a, code)
+
+
+# ---------------------------------------------------------------- level 1
+
+def _sym_quant(kind, X):
+    if kind == "act":
+        return oracle.quantize_act(X) + (127,)
+    return oracle.quantize_weights_i8(X) + (119,)
+
+
+@pytest.mark.parametrize("kind", ["act", "w"])
+def test_symmetric_int8_properties(kind):
+    rng = np.random.default_rng(1)
+    X = (rng.standard_normal((37, 200)) * rng.uniform(0.01, 10, (37, 1))).astype(np.float32)
+    X[5] = 0.0
+    Q, s, R = _sym_quant(kind, X)
+    assert Q.dtype == np.int8 and s.dtype == np.float32
+    assert np.abs(Q.astype(int)).max() <= R
+    # the absmax element of each nonzero row lands exactly on +-R
+    nz = np.abs(X).max(1) > 0
+    assert np.all(np.abs(Q[nz].astype(int)).max(1) == R)
+    # zero row: zero scale and zero codes
+    assert s[5] == 0 and not Q[5].any()
+    # scale is absmax / R in fp32
+    assert np.array_equal(s, (np.abs(X).max(1) / np.float32(R)).astype(np.float32))
+    # rounding error at most half a step
+    err = np.abs(X.astype(np.float64) - s[:, None].astype(np.float64) * Q)
+    assert np.all(err <= 0.5 * s[:, None] * (1 + 1e-6) + 1e-30)
+    # odd symmetry
+    Qn, sn, _ = _sym_quant(kind, -X)
+    assert np.array_equal(Qn, -Q) and np.array_equal(sn, s)
+    # power-of-two scale invariance
+    Q4, s4, _ = _sym_quant(kind, X * 4)
+    assert np.array_equal(Q4, Q) and np.array_equal(s4, s * 4)
+    # monotone along a row
+    order = np.argsort(X[0], kind="stable")
+    assert np.all(np.diff(Q[0][order].astype(int)) >= 0)
+    # rows are independent and not transposed
+    perm = rng.permutation(37)
+    Qp, sp, _ = _sym_quant(kind, X[perm])
+    assert np.array_equal(Qp, Q[perm]) and np.array_equal(sp, s[perm])
+
+
+def test_round_half_to_even_ties():
+    """Reading R3: FP -> INT8 rounds half to even.  With absmax 127 the
+    activation scale is exactly 1.0, so x/s = x and ties are exact."""
+    X = np.array([[127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -0.5, 126.5]], np.float32)
+    Q, s = oracle.quantize_act(X)
+    assert s[0] == 1.0
+    assert list(Q[0]) == [127, 2, 4, -2, -4, 0, 2, 0, 126]
+
+
+def test_weight_end_to_end_error_bound():
+    """|W - s_w * (code*s_u8 + min)| <= s_w * (1/2 + s_u8/2): half a step of
+    level 1 plus half a group step of level 2 (ceil rule)."""
+    rng = np.random.default_rng(2)
+    W = (rng.standard_normal((48, 512)) * 0.02).astype(np.float32)
+    W[3, 64:128] = 0.01          # constant group
+    W[7] = 0                     # zero channel
+    wq = oracle.quantize_weights(W, want_i8=True)
+    W8 = oracle.dequant_weights(wq["codes"], wq["s_u8"], wq["a"])
+    smul = np.repeat(wq["s_u8"].astype(np.float64), 64, axis=1)
+    bound = wq["s_w"][:, None].astype(np.float64) * (0.5 + smul / 2) * (1 + 1e-6)
+    err = np.abs(W.astype(np.float64) - wq["s_w"][:, None] * W8.astype(np.float64))
+    assert np.all(err <= bound + 1e-30)
+    assert not W8[7].any() and wq["s_w"][7] == 0
+    # constant group reconstructs its INT8 value exactly
+    assert np.all(W8[3, 64:128] == wq["q_i8"][3, 64:128])
+    # groups are along K within one channel: changing one group's values
+    # changes only that group's (s_u8, a)
+    W2 = W.copy()
+    W2[10, 192:256] *= 0.5
+    wq2 = oracle.quantize_weights(W2)
+    diff = (wq2["s_u8"] != wq["s_u8"]) | (wq2["a"] != wq["a"])
+    assert set(zip(*np.nonzero(diff))) <= {(10, 3)}
+
+
+# ------------------------------------------------------------------- GEMM
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 64), (2, 3, 64), (4, 2, 128), (3, 4, 192)])
+def test_gemm_bruteforce_tiny(M, N, K):
+    rng = np.random.default_rng(M * 100 + N * 10 + K)
+    X = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    W = rng.integers(-119, 128, (N, K)).astype(np.int8)
+    acc = oracle.gemm_i32(X, W)
+    for m, n in itertools.product(range(M), range(N)):
+        ref = 0
+        for k in range(K):
+            ref += int(X[m, k]) * int(W[n, k])
+        assert acc[m, n] == ref
+
+
+def test_gemm_against_numpy_int64_and_extremes():
+    rng = np.random.default_rng(3)
+    X = rng.integers(-127, 128, (33, 320)).astype(np.int8)
+    W = rng.integers(-119, 128, (70, 320)).astype(np.int8)
+    acc = oracle.gemm_i32(X, W)
+    assert acc.shape == (33, 70)
+    assert np.array_equal(acc, X.astype(np.int64) @ W.astype(np.int64).T)
+    K = 28672
+    Xm = np.full((2, K), 127, np.int8)
+    Xm[1] = -127
+    Wm = np.full((1, K), 127, np.int8)
+    acc = oracle.gemm_i32(Xm, Wm)
+    assert acc[0, 0] == K * 127 * 127 and acc[1, 0] == -K * 127 * 127
+
+
+def test_fp64_dequantize_then_matmul_agrees():
+    """sum_k (s_x Qx)(s_w W8) in float64 equals s_x s_w acc (R6 before the
+    bf16 rounding), and the bf16 output is that value rounded once."""
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((24, 256)).astype(np.float32)
+    W = (rng.standard_normal((40, 256)) * 0.02).astype(np.float32)
+    Xq, s_x = oracle.quantize_act(X)
+    wq = oracle.quantize_weights(W)
+    acc, Y = oracle.w4a8_gemm(Xq, s_x, wq)
+    W8 = oracle.dequant_weights(wq["codes"], wq["s_u8"], wq["a"])
+    Y64 = (Xq * s_x[:, None].astype(np.float64)) @ (W8 * wq["s_w"][:, None].astype(np.float64)).T
+    Yacc = s_x[:, None].astype(np.float64) * wq["s_w"][None, :].astype(np.float64) * acc
+    # float64 summation error is relative to the sum of |terms|
+    mag = (np.abs(Xq) * s_x[:, None].astype(np.float64)) @ (np.abs(W8) * wq["s_w"][:, None].astype(np.float64)).T
+    assert np.all(np.abs(Y64 - Yacc) <= 1e-13 * mag)
+    Yf = oracle.bf16_bits_to_float(Y).astype(np.float64)
+    # one rounding to bf16: relative error at most 2^-9 (half an ulp)
+    nz = Yacc != 0
+    assert np.all(np.abs(Yf[nz] - Yacc[nz]) <= np.abs(Yacc[nz]) * 2.0 ** -8)
+    # and within the propagated quantization error of the unquantized product
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    errW = wq["s_w"][:, None] * (0.5 + np.repeat(wq["s_u8"], 64, axis=1) / 2.0)
+    errX = np.broadcast_to(s_x[:, None] / 2.0, X.shape)
+    What = W8 * wq["s_w"][:, None].astype(np.float64)
+    bound = np.abs(X) @ errW.T + errX @ np.abs(What).T
+    assert np.all(np.abs(Y64 - ref) <= bound * (1 + 1e-9))
+    # sampled entry point agrees with the full one
+    ms = np.array([0, 23, 5, 11]); ns = np.array([0, 39, 17, 2])
+    a2, y2 = oracle.w4a8_gemm_sampled(Xq, s_x, wq, ms, ns)
+    assert np.array_equal(a2, acc[ms, ns]) and np.array_equal(y2, Y[ms, ns])
+
+
+# ------------------------------------------------------------- bf16 RNE
+
+def test_bf16_rounding_hand_cases():
+    b = oracle.bf16_from_double
+    assert b(1.0) == 0x3F80
+    assert b(-2.0) == 0xC000
+    assert b(1 + 2 ** -8) == 0x3F80              # tie -> even
+    assert b(1 + 3 * 2 ** -8) == 0x3F82          # tie -> even (up)
+    assert b(1 + 2 ** -8 + 2 ** -40) == 0x3F81   # one rounding, not via fp32
+    assert b(0.0) == 0x0000
+    assert b((2 - 2 ** -7) * 2.0 ** 127) == 0x7F7F
+    assert b(2.0 ** 128) == 0x7F80
+    assert b(-(2.0 ** 129)) == 0xFF80
+    assert b(2.0 ** -126) == 0x0080
+    assert b(2.0 ** -130) == 0x0008
+    assert b((2 - 2 ** -8) * 2.0 ** 127 * (1 - 2 ** -30)) == 0x7F7F
+
+
+def test_bf16_rounding_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(20000) * np.exp2(rng.integers(-60, 60, 20000))).astype(np.float32)
+    ours = np.array([oracle.bf16_from_double(float(v)) for v in x], np.uint16)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_epilogue_scales_and_signs():
+    acc = np.array([[3, -3, 0], [1000, -7, 2 ** 20]], np.int32)
+    s_x = np.array([0.5, 2.0], np.float32)
+    s_w = np.array([0.25, 1.0, 4.0], np.float32)
+    Y = oracle.bf16_bits_to_float(oracle.epilogue_bf16(acc, s_x, s_w))
+    ref = (s_x[:, None].astype(np.float64) * s_w[None] * acc).astype(np.float32)
+    assert np.array_equal(Y, torch.from_numpy(ref).to(torch.bfloat16).float().numpy())
