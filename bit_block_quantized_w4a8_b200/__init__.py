@@ -1,0 +1,247 @@
+"""B200-native block-quantized W4A8 GEMM (LiquidQuant-style INT4 weights,
+per-token INT8 activations, tcgen05 INT8 tensor cores, bf16 output).
+
+This module is the Python binding of ``libw4a8.so`` (C ABI in
+``include/w4a8.h``).  It only marshals arguments: every step of the path runs
+in the library's CUDA kernels.  PyTorch provides device memory and streams.
+The functions carry the names of the C entry points; all tensors are CUDA
+tensors on the current device and work is enqueued on the current stream
+unless ``stream`` is given.
+
+If the library has not been built, every call raises ``W4A8Error``; there is
+no fallback implementation.
+"""
+import ctypes as _ct
+import os as _os
+import threading as _threading
+
+import torch as _torch
+
+from .build import LIB as _LIB_PATH
+
+__all__ = [
+    "W4A8Error", "lib", "w4a8_version", "w4a8_status_string",
+    "w4a8_packed_weight_bytes", "w4a8_quantize_weights", "w4a8_unpack_weights",
+    "w4a8_quantize_act", "w4a8_gemm_workspace_bytes", "w4a8_workspace_init",
+    "w4a8_gemm", "w4a8_gemm_i32", "w4a8_gemm_schedule", "w4a8_get_status",
+    "w4a8_debug_timeout_probe", "PackedWeights", "workspace_for",
+]
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED_SHAPE = -2
+ERR_MISALIGNED = -3
+ERR_WORKSPACE = -4
+ERR_CUDA = -5
+ERR_TIMEOUT = -6
+ERR_BAD_PACKED = -7
+
+
+class W4A8Error(RuntimeError):
+    def __init__(self, what, code):
+        super().__init__("%s failed: %s (%d)" % (what, w4a8_status_string(code), code))
+        self.code = code
+
+
+_lib = None
+_lock = _threading.Lock()
+
+
+def lib():
+    """The loaded ``libw4a8.so`` (ctypes.CDLL)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not _os.path.exists(_LIB_PATH):
+            raise W4A8Error("loading %s (not built; run `python -m "
+                            "bit_block_quantized_w4a8_b200.build`)" % _LIB_PATH,
+                            ERR_CUDA)
+        L = _ct.CDLL(_LIB_PATH)
+        i32, sz, p, ll = _ct.c_int, _ct.c_size_t, _ct.c_void_p, _ct.c_longlong
+        sigs = {
+            "w4a8_status_string": ([i32], _ct.c_char_p),
+            "w4a8_version": ([], i32),
+            "w4a8_packed_weight_bytes": ([i32, i32, i32], sz),
+            "w4a8_quantize_weights": ([p, i32, i32, i32, p, p], i32),
+            "w4a8_unpack_weights": ([p, i32, i32, p, p, p, p, p], i32),
+            "w4a8_quantize_act": ([p, i32, i32, p, p, p], i32),
+            "w4a8_gemm_workspace_bytes": ([i32, i32, i32], sz),
+            "w4a8_workspace_init": ([p, sz, p], i32),
+            "w4a8_gemm": ([p, p, p, i32, i32, i32, p, p, sz, p], i32),
+            "w4a8_gemm_i32": ([p, p, i32, i32, i32, p, p, sz, p], i32),
+            "w4a8_gemm_schedule": ([i32, i32, i32, p, p, p], i32),
+            "w4a8_get_status": ([p], i32),
+            "w4a8_debug_timeout_probe": ([ll, p], i32),
+        }
+        for name, (args, res) in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else _ct.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = _torch.cuda.current_stream()
+    return _ct.c_void_p(stream.cuda_stream)
+
+
+def _check(rc, what):
+    if rc != OK:
+        raise W4A8Error(what, rc)
+
+
+def _need(t, dtype, ndim, name):
+    if not isinstance(t, _torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype or t.dim() != ndim or not t.is_contiguous():
+        raise TypeError("%s must be a contiguous %dD %s tensor" % (name, ndim, dtype))
+
+
+def w4a8_status_string(code):
+    return lib().w4a8_status_string(int(code)).decode()
+
+
+def w4a8_version():
+    return lib().w4a8_version()
+
+
+def w4a8_packed_weight_bytes(N, K, group=64):
+    return int(lib().w4a8_packed_weight_bytes(int(N), int(K), int(group)))
+
+
+class PackedWeights:
+    """A packed LQQ weight buffer (uint8 CUDA tensor) with its shape."""
+
+    def __init__(self, data, N, K, group):
+        self.data, self.N, self.K, self.group = data, int(N), int(K), int(group)
+
+    def __repr__(self):
+        return "PackedWeights(N=%d, K=%d, group=%d, bytes=%d)" % (
+            self.N, self.K, self.group, self.data.numel())
+
+
+def w4a8_quantize_weights(W, group=64, out=None, stream=None):
+    """Quantize fp32 weights W [N, K] into a packed LQQ buffer."""
+    _need(W, _torch.float32, 2, "W")
+    N, K = W.shape
+    nbytes = w4a8_packed_weight_bytes(N, K, group)
+    if nbytes == 0:
+        raise W4A8Error("w4a8_packed_weight_bytes", ERR_UNSUPPORTED_SHAPE)
+    if out is None:
+        out = _torch.empty(nbytes, dtype=_torch.uint8, device=W.device)
+    elif out.numel() < nbytes or out.dtype != _torch.uint8:
+        raise ValueError("out must be a uint8 tensor of at least %d bytes" % nbytes)
+    _check(lib().w4a8_quantize_weights(_ptr(W), N, K, group, _ptr(out), _stream(stream)),
+           "w4a8_quantize_weights")
+    return PackedWeights(out, N, K, group)
+
+
+def w4a8_unpack_weights(packed, stream=None):
+    """Canonical arrays of a packed buffer: codes [N,K], s_u8 [N,G], a [N,G], s_w [N]."""
+    d = packed.data.device
+    N, K, G = packed.N, packed.K, packed.K // packed.group
+    codes = _torch.empty(N, K, dtype=_torch.uint8, device=d)
+    s = _torch.empty(N, G, dtype=_torch.uint8, device=d)
+    a = _torch.empty(N, G, dtype=_torch.uint8, device=d)
+    sw = _torch.empty(N, dtype=_torch.float32, device=d)
+    _check(lib().w4a8_unpack_weights(_ptr(packed.data), N, K, _ptr(codes), _ptr(s), _ptr(a),
+                                     _ptr(sw), _stream(stream)), "w4a8_unpack_weights")
+    return dict(codes=codes, s_u8=s, a=a, s_w=sw)
+
+
+def w4a8_quantize_act(X, out=None, scale_out=None, stream=None):
+    """Per-token INT8 quantization of fp32 X [M, K]: returns (Xq int8, s_x fp32)."""
+    _need(X, _torch.float32, 2, "X")
+    M, K = X.shape
+    Xq = out if out is not None else _torch.empty(M, K, dtype=_torch.int8, device=X.device)
+    sx = scale_out if scale_out is not None else _torch.empty(M, dtype=_torch.float32,
+                                                              device=X.device)
+    _check(lib().w4a8_quantize_act(_ptr(X), M, K, _ptr(Xq), _ptr(sx), _stream(stream)),
+           "w4a8_quantize_act")
+    return Xq, sx
+
+
+def w4a8_gemm_workspace_bytes(M, N, K):
+    return int(lib().w4a8_gemm_workspace_bytes(int(M), int(N), int(K)))
+
+
+def w4a8_workspace_init(ws, stream=None):
+    _check(lib().w4a8_workspace_init(_ptr(ws), ws.numel(), _stream(stream)),
+           "w4a8_workspace_init")
+
+
+_ws_cache = {}
+
+
+def workspace_for(M, N, K, device=None, stream=None):
+    """A zero-filled workspace big enough for (M, N, K), cached per device and
+    stream (calls on one stream run in order, so they may share it)."""
+    need = w4a8_gemm_workspace_bytes(M, N, K)
+    if need == 0:
+        return None
+    dev = _torch.device(device) if device is not None else _torch.device(
+        "cuda", _torch.cuda.current_device())
+    s = stream if stream is not None else _torch.cuda.current_stream(dev)
+    key = (dev.index, s.cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = _torch.zeros(max(need, 1 << 20), dtype=_torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    return ws
+
+
+def w4a8_gemm(Xq, s_x, packed, out=None, workspace=None, stream=None):
+    """Y [M, N] bf16 = (s_x[m] s_w[n]) * sum_k Xq[m,k] Wdq[n,k]."""
+    _need(Xq, _torch.int8, 2, "Xq")
+    _need(s_x, _torch.float32, 1, "s_x")
+    M, K = Xq.shape
+    if K != packed.K:
+        raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
+    N = packed.N
+    Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
+    ws = workspace if workspace is not None else workspace_for(M, N, K, Xq.device, stream)
+    _check(lib().w4a8_gemm(_ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y), _ptr(ws),
+                           0 if ws is None else ws.numel(), _stream(stream)), "w4a8_gemm")
+    return Y
+
+
+def w4a8_gemm_i32(Xq, packed, out=None, workspace=None, stream=None):
+    """Exact INT32 accumulators acc [M, N] = sum_k Xq[m,k] Wdq[n,k]."""
+    _need(Xq, _torch.int8, 2, "Xq")
+    M, K = Xq.shape
+    if K != packed.K:
+        raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
+    N = packed.N
+    acc = out if out is not None else _torch.empty(M, N, dtype=_torch.int32, device=Xq.device)
+    ws = workspace if workspace is not None else workspace_for(M, N, K, Xq.device, stream)
+    _check(lib().w4a8_gemm_i32(_ptr(Xq), _ptr(packed.data), M, N, K, _ptr(acc), _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream(stream)),
+           "w4a8_gemm_i32")
+    return acc
+
+
+def w4a8_gemm_schedule(M, N, K):
+    """(tokens per tile, split-K factor, CTAs) the library picks for a shape."""
+    t, s, c = _ct.c_int(0), _ct.c_int(0), _ct.c_int(0)
+    _check(lib().w4a8_gemm_schedule(int(M), int(N), int(K), _ct.byref(t), _ct.byref(s),
+                                    _ct.byref(c)), "w4a8_gemm_schedule")
+    return t.value, s.value, c.value
+
+
+def w4a8_get_status(stream=None):
+    """Synchronize the stream and return/clear the device status word."""
+    return lib().w4a8_get_status(_stream(stream))
+
+
+def w4a8_debug_timeout_probe(limit_ns, stream=None):
+    _check(lib().w4a8_debug_timeout_probe(int(limit_ns), _stream(stream)),
+           "w4a8_debug_timeout_probe")

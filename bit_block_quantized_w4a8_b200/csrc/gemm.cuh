@@ -1,0 +1,334 @@
+// gemm.cuh -- the W4A8 GEMM for sm_100a: packed LQQ INT4 weights are
+// dequantized to INT8 by CUDA-core warps straight into tensor memory (TMEM)
+// and multiplied with INT8 activations by tcgen05.mma kind::i8 (INT32
+// accumulators in TMEM), then a fused epilogue applies s_x[m] * s_w[n] and
+// stores bf16 (or the exact INT32 accumulators).
+//
+// Method (review page "LiquidGEMM", pith.science verdict on arXiv
+// 2509.01229): dequantization (q_u4 * s_u8 + a) XOR 0x80, two integer
+// instructions per four weights after unpacking, never leaving UINT8
+// (key_machinery; referee summary; referee minor 1, paper Sec. 5.3); the
+// INT8 x INT8 tensor-core product with INT32 accumulation (lead); a
+// producer / several-consumer pipeline that overlaps loading, CUDA-core
+// dequantization and tensor-core MMA (key_machinery, "ImFP").
+//
+// The B200 design (not the page's Hopper design):
+//   * MMA orientation: the 128 weight rows of a tile are the MMA's M
+//     dimension and live in TMEM as the A operand (tcgen05.mma with A from
+//     tensor memory); the T tokens of the tile are the MMA's N dimension
+//     (B operand, shared memory, 128-byte swizzle, loaded by TMA).  The
+//     dequantized weights therefore never touch shared memory: one
+//     tcgen05.st per 32 weights and thread.
+//   * Warp roles per CTA: warp 0 issues the copies (1-D bulk copy of a
+//     packed weight tile + 2-D TMA of the activation tile), warp 1 issues
+//     the MMAs (one thread), DQG groups of 4 warps dequantize (thread =
+//     weight row = TMEM lane) and then run the epilogue.
+//   * Ring of STAGES slots, each holding one weight tile and one
+//     activation tile in shared memory and one 32-column A slot in TMEM.
+//     Barriers per slot: full (copies landed), dq (A slot written), empty
+//     (MMAs that read the slot completed, via tcgen05.commit).
+//   * Split-K for few output tiles (decode): each split adds its INT32
+//     partials into a workspace with red.add; the last split to arrive (a
+//     per-tile counter) applies the epilogue and zeroes what it used.
+//   * Every wait is bounded (globaltimer); a wait that runs out records a
+//     timeout in the device status word and all roles leave their loops,
+//     wait for their own copies / MMAs in flight, free TMEM and return.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "layout.cuh"
+#include "ptx.cuh"
+
+namespace w4a8 {
+
+struct GemmParams {
+  const uint8_t* tiles;   // packed weight tiles
+  const float* s_w;       // packed per-channel scales [n_pad]
+  const float* s_x;       // per-token scales [M] (bf16 output only)
+  uint16_t* Y;            // [M][N] bf16 bits, or nullptr
+  int32_t* acc;           // [M][N] int32, or nullptr
+  int32_t* ws;            // split-K partials [m_tiles][n_pad][T]
+  uint32_t* counters;     // split-K arrivals [m_tiles][n_tiles]
+  int M, N, K, n_pad;
+  int kt_total;           // K / 128
+  int splits, kt_per_split;
+  int n_tiles, m_tiles;
+  unsigned long long wait_limit_ns;
+  const PackedHeader* hdr;  // checked against (N, K) before any store
+};
+
+template <int T, int STAGES, int DQG>
+struct GemmCfg {
+  static_assert(T % 16 == 0 && T >= 16 && T <= 256, "MMA N for M=128");
+  static constexpr int kXBytes = T * kTileK;             // activation tile
+  static constexpr int kStageBytes = kXBytes + kTileBytes;
+  static constexpr int kThreads = (2 + 4 * DQG) * 32;
+  static constexpr int kA0 = T < 32 ? 32 : T;             // first A column
+  static constexpr int kColsUsed = kA0 + 32 * STAGES;
+  static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
+                                   : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
+  static_assert(kColsUsed <= 512, "TMEM columns");
+  // shared memory: x tiles | w tiles | barriers | misc | s_x cache
+  static constexpr int kOffW = STAGES * kXBytes;
+  static constexpr int kOffBar = kOffW + STAGES * kTileBytes;
+  static constexpr int kNumBars = 3 * STAGES + 1;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kOffSx = kOffMisc + 16;
+  static constexpr int kSmemBytes = kOffSx + 4 * T + 1024;  // + alignment slack
+  static constexpr uint32_t kTxBytes = kXBytes + kTileBytes;
+};
+
+// Dequantize four packed words (32 codes of one row, k order given by the
+// packed layout) with the group's integer scale s and offset a into eight
+// words of four INT8 values each: (code * s + a) XOR 0x80 per byte.
+__device__ __forceinline__ void dequant_chunk(uint4 v, uint32_t s, uint32_t a4,
+                                              uint32_t (&out)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t lo = w[j] & 0x0F0F0F0Fu;
+    const uint32_t hi = (w[j] >> 4) & 0x0F0F0F0Fu;
+    out[2 * j] = (lo * s + a4) ^ 0x80808080u;
+    out[2 * j + 1] = (hi * s + a4) ^ 0x80808080u;
+  }
+}
+
+// All 32 lanes wait; the warp proceeds only if every lane saw the phase
+// complete (keeps the .sync.aligned tcgen05 instructions warp-uniform).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
+                                          volatile int* abort, uint64_t lim) {
+  const bool ok = mbar_wait(bar, parity, abort, lim);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int T, int STAGES, int DQG, int MINB>
+__global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
+    w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                     const GemmParams p) {
+  using C = GemmCfg<T, STAGES, DQG>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const uint32_t bar_full = sbase + C::kOffBar;        // + 8 s
+  const uint32_t bar_empty = bar_full + 8 * STAGES;    // + 8 s
+  const uint32_t bar_dq = bar_empty + 8 * STAGES;      // + 8 s
+  const uint32_t bar_acc = bar_dq + 8 * STAGES;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
+  volatile int* ep_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
+  float* sx_s = reinterpret_cast<float*>(smem + C::kOffSx);
+
+  // tile coordinates: channel block fastest, then token block, then split
+  const int n_tile = blockIdx.x % p.n_tiles;
+  const int rest = blockIdx.x / p.n_tiles;
+  const int m_tile = rest % p.m_tiles;
+  const int split = rest / p.m_tiles;
+  const int kt0 = split * p.kt_per_split;
+  const int kt1 = min(kt0 + p.kt_per_split, p.kt_total);
+  const int nk = kt1 - kt0;
+  const int m0 = m_tile * T;
+  const uint64_t lim = p.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_dq + 8 * s, 4);
+    }
+    mbar_init(bar_acc, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (p.Y) {
+    for (int i = threadIdx.x; i < T; i += C::kThreads)
+      sx_s[i] = (m0 + i < p.M) ? p.s_x[m0 + i] : 0.0f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_x);
+      const uint64_t pol = l2_policy_evict_first();
+      const uint8_t* wsrc = p.tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
+      int issued = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
+        mbar_arrive_expect_tx(bar_full + 8 * s, C::kTxBytes);
+        bulk_g2s(sbase + C::kOffW + s * kTileBytes, wsrc + (size_t)it * kTileBytes,
+                 kTileBytes, bar_full + 8 * s, pol);
+        tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
+                    bar_full + 8 * s);
+        issued = it + 1;
+      }
+      if (*abort_flag) {
+        // let the copies already issued land before the CTA goes away
+        for (int it = issued - STAGES < 0 ? 0 : issued - STAGES; it < issued; ++it)
+          mbar_wait(bar_full + 8 * (it % STAGES), (it / STAGES) & 1, nullptr, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(128, T);
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(bar_dq + 8 * s, ph, abort_flag, lim)) break;
+        if (!mbar_wait(bar_full + 8 * s, ph, abort_flag, lim)) break;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + C::kA0 + 32 * s;
+        const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 32; ++kk)
+          mma_i8_ts(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc,
+                    (it | kk) != 0);
+        tc_commit(bar_empty + 8 * s);
+      }
+      tc_commit(bar_acc);  // also on abort: tracks every MMA issued
+    }
+  } else {
+    // --------------------------------------------- dequantization warps
+    const int dg = (warp - 2) / 4;         // dequant group
+    const int quarter = warp & 3;          // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;     // weight row in the tile = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    for (int it = dg; it < nk; it += DQG) {
+      const int s = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      if (!warp_wait(bar_full + 8 * s, ph, abort_flag, lim)) break;
+      // the MMAs of the previous round of this slot are done (TMEM A free)
+      if (!warp_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
+      tc_fence_after();
+      const uint32_t wbase = sbase + C::kOffW + s * kTileBytes;
+      const uint32_t prm = lds32(wbase + kCodeBytes + 4 * r);
+      const uint32_t a_col = lane_base + C::kA0 + 32 * s;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t sh = (c < 2) ? 0 : 16;
+        const uint32_t sc = (prm >> sh) & 0xFFu;
+        const uint32_t a4 = ((prm >> (sh + 8)) & 0xFFu) * 0x01010101u;
+        const uint4 v = lds128(wbase + (c * kTileN + r) * 16);
+        uint32_t out[8];
+        dequant_chunk(v, sc, a4, out);
+        tmem_st_x8(a_col + 8 * c, out);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dq + 8 * s);
+    }
+
+    // -------------------------------------------------------- epilogue
+    const int nthr = 128 * DQG;
+    bool hdr_ok = true;
+    if (warp == 2 && lane == 0)
+      hdr_ok = p.hdr->magic == kMagic && p.hdr->N == p.N && p.hdr->K == p.K;
+    warp_wait(bar_acc, 0, abort_flag, lim);
+    tc_fence_after();
+    // one thread turns the abort flag into a value every epilogue thread
+    // reads between the same two barriers, so the branch below is uniform
+    named_bar_sync(1, nthr);
+    if (warp == 2 && lane == 0) {
+      if (!hdr_ok) record_status(kDevBadPacked);
+      *ep_flag = (*abort_flag || !hdr_ok) ? 0 : 1;
+    }
+    named_bar_sync(1, nthr);
+    const int n = n_tile * kTileN + r;
+    if (*ep_flag) {
+      if (p.splits == 1) {
+        const float swn = n < p.N ? p.s_w[n] : 0.0f;
+        for (int j = dg; j < T / 16; j += DQG) {
+          uint32_t v[16];
+          tmem_ld_x16(lane_base + 16 * j, v);
+          tmem_wait_ld();
+          if (n < p.N) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              const int m = m0 + 16 * j + t;
+              if (m < p.M) {
+                const int32_t a = (int32_t)v[t];
+                if (p.Y) {
+                  const float y = (float)a * (sx_s[16 * j + t] * swn);
+                  p.Y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+                } else {
+                  p.acc[(size_t)m * p.N + n] = a;
+                }
+              }
+            }
+          }
+        }
+      } else {
+        int32_t* wrow = p.ws + ((size_t)m_tile * p.n_pad + n) * T;
+        for (int j = dg; j < T / 16; j += DQG) {
+          uint32_t v[16];
+          tmem_ld_x16(lane_base + 16 * j, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (m0 + 16 * j + t < p.M) red_add_s32(wrow + 16 * j + t, (int32_t)v[t]);
+        }
+        __threadfence();
+        named_bar_sync(1, nthr);
+        uint32_t* cnt = p.counters + (size_t)m_tile * p.n_tiles + n_tile;
+        if (warp == 2 && lane == 0) {
+          const uint32_t old = atomicAdd(cnt, 1u);
+          *last_flag = (old == (uint32_t)(p.splits - 1)) ? 1 : 0;
+        }
+        named_bar_sync(1, nthr);
+        if (*last_flag) {
+          __threadfence();
+          const float swn = n < p.N ? p.s_w[n] : 0.0f;
+          for (int j = dg; j < T / 16; j += DQG) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              const int m = m0 + 16 * j + t;
+              if (m < p.M) {
+                const int32_t a = __ldcg(wrow + 16 * j + t);
+                __stcg(wrow + 16 * j + t, 0);
+                if (n < p.N) {
+                  if (p.Y) {
+                    const float y = (float)a * (sx_s[16 * j + t] * swn);
+                    p.Y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+                  } else {
+                    p.acc[(size_t)m * p.N + n] = a;
+                  }
+                }
+              }
+            }
+          }
+          if (warp == 2 && lane == 0) *cnt = 0u;
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  if (threadIdx.x == 0 && *abort_flag) {
+    // every MMA issued has completed before TMEM is released
+    mbar_wait(bar_acc, 0, nullptr, lim);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace w4a8

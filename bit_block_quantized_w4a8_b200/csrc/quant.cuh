@@ -1,0 +1,220 @@
+// quant.cuh -- offline LQQ weight quantization + packing, its inverse (a
+// test aid), and per-token INT8 activation quantization.
+//
+// Method: review page "LiquidGEMM" (pith.science verdict on arXiv
+// 2509.01229): level-1 per-channel INT8 in the protective range +-119 and
+// the integer group scale s_u8 <= 16 (referee major 3, paper Sec. 4 Eq. 7);
+// shift by the group minimum into UINT8, UINT4 codes rounded to nearest
+// (referee summary; referee minor 2, Sec. 4 Eq. 10); offset a = 2^7 + min
+// (key_machinery); per-token INT8 activations (supporting citation [29]).
+//
+// Every FP -> integer decision uses IEEE fp32 division (__fdiv_rn, never a
+// reciprocal) and round-half-to-even (__float2int_rn), so codes are exactly
+// reproducible on any IEEE machine.
+#pragma once
+#include <cstdint>
+#include "layout.cuh"
+
+namespace w4a8 {
+
+__device__ __forceinline__ int quant_sym(float x, float s, int range) {
+  if (s == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(x, s));
+  return q > range ? range : (q < -range ? -range : q);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// One warp per output channel: s_w[n] = absmax / 119, written straight into
+// the packed buffer (padding channels get 0).  Block 0 also writes the header.
+__global__ void __launch_bounds__(256) weight_scale_kernel(
+    const float* __restrict__ W, int N, int K, int group, int n_pad,
+    uint8_t* __restrict__ packed) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  float* s_w = reinterpret_cast<float*>(packed + sw_offset_bytes());
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    PackedHeader h;
+    h.magic = kMagic;
+    h.version = kLayoutVersion;
+    h.N = N;
+    h.K = K;
+    h.group = group;
+    h.n_pad = n_pad;
+    h.sw_offset = sw_offset_bytes();
+    h.tiles_offset = tiles_offset_bytes(n_pad);
+    h.total_bytes = packed_bytes(N, K);
+    *reinterpret_cast<PackedHeader*>(packed) = h;
+  }
+  if (warp >= n_pad) return;
+  float amax = 0.0f;
+  if (warp < N) {
+    const float4* row = reinterpret_cast<const float4*>(W + (size_t)warp * K);
+    for (int i = lane; i < K / 4; i += 32) {
+      float4 v = __ldg(row + i);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)),
+                               fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    amax = warp_max(amax);
+  }
+  if (lane == 0) s_w[warp] = __fdiv_rn(amax, 119.0f);
+}
+
+// One CTA (128 threads) per tile of 128 channels x 128 k.  The fp32 tile is
+// staged through shared memory (row stride 129 floats: conflict-free) so the
+// global reads are coalesced; thread r then owns channel 128 nb + r.
+constexpr int kPackSmemBytes = kTileN * (kTileK + 1) * 4;
+
+__global__ void __launch_bounds__(128) weight_pack_kernel(
+    const float* __restrict__ W, int N, int K, int group, int n_pad,
+    uint8_t* __restrict__ packed) {
+  extern __shared__ float tile[];  // [128][129]
+  const int kb = blockIdx.x, nb = blockIdx.y, r = threadIdx.x;
+  const int kt_total = K / kTileK;
+  const float* s_w = reinterpret_cast<const float*>(packed + sw_offset_bytes());
+  uint8_t* dst = packed + tiles_offset_bytes(n_pad) +
+                 ((size_t)nb * kt_total + kb) * kTileBytes;
+  // coalesced load: 32 consecutive threads read 32 consecutive floats
+  for (int e = r; e < kTileN * kTileK; e += 128) {
+    int row = e / kTileK, col = e % kTileK;
+    int n = nb * kTileN + row;
+    tile[row * (kTileK + 1) + col] =
+        n < N ? __ldg(W + (size_t)n * K + (size_t)kb * kTileK + col) : 0.0f;
+  }
+  __syncthreads();
+  const int n = nb * kTileN + r;
+  const float s = s_w[n];
+  const float* x = tile + r * (kTileK + 1);
+  // level 1 then level 2, per group of `group` (64 or 128) k-values
+  uint8_t sg[2], ag[2];
+  int mnv[2];
+  const int ng = kTileK / 64;  // two parameter slots per tile row
+  for (int h = 0; h < ng; ++h) {
+    const int g0 = (group == 128) ? 0 : h * 64, glen = group;
+    int mn = 127, mx = -127;
+    for (int i = 0; i < glen; ++i) {
+      int q = quant_sym(x[g0 + i], s, 119);
+      mn = min(mn, q);
+      mx = max(mx, q);
+    }
+    int sc = (mx - mn + 14) / 15;  // ceil((max - min) / 15)
+    sc = sc < 1 ? 1 : sc;
+    if (n >= N) {  // padding channel: dequantizes to 0
+      sc = 1;
+      mn = 0;
+    }
+    sg[h] = (uint8_t)sc;
+    ag[h] = (uint8_t)(128 + mn);
+    mnv[h] = mn;
+  }
+  uint32_t prm = (uint32_t)sg[0] | ((uint32_t)ag[0] << 8) |
+                 ((uint32_t)sg[1] << 16) | ((uint32_t)ag[1] << 24);
+  *reinterpret_cast<uint32_t*>(dst + kCodeBytes + 4 * r) = prm;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    const int h = c / 2;
+    const int sc = sg[h], mn = mnv[h];
+    uint32_t words[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int k_lo = 32 * c + 8 * j + b, k_hi = k_lo + 4;
+        int c_lo = 0, c_hi = 0;
+        if (n < N) {
+          c_lo = (2 * (quant_sym(x[k_lo], s, 119) - mn) + sc) / (2 * sc);
+          c_hi = (2 * (quant_sym(x[k_hi], s, 119) - mn) + sc) / (2 * sc);
+        }
+        w |= (uint32_t)(c_lo | (c_hi << 4)) << (8 * b);
+      }
+      words[j] = w;
+    }
+    *reinterpret_cast<uint4*>(dst + (c * kTileN + r) * 16) =
+        make_uint4(words[0], words[1], words[2], words[3]);
+  }
+}
+
+// Inverse of the packing (test aid): canonical codes / s_u8 / a / s_w.
+__global__ void __launch_bounds__(128) weight_unpack_kernel(
+    const uint8_t* __restrict__ packed, int N, int K, int n_pad,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ s_u8,
+    uint8_t* __restrict__ a, float* __restrict__ s_w_out) {
+  const int kb = blockIdx.x, nb = blockIdx.y, r = threadIdx.x;
+  const int kt_total = K / kTileK;
+  const int n = nb * kTileN + r;
+  if (n >= N) return;
+  const uint8_t* src = packed + tiles_offset_bytes(n_pad) +
+                       ((size_t)nb * kt_total + kb) * kTileBytes;
+  const uint32_t prm = *reinterpret_cast<const uint32_t*>(src + kCodeBytes + 4 * r);
+  const int group = reinterpret_cast<const PackedHeader*>(packed)->group;
+  const int G = K / group;
+  if (group == 64) {
+    s_u8[(size_t)n * G + 2 * kb] = prm & 0xFF;
+    a[(size_t)n * G + 2 * kb] = (prm >> 8) & 0xFF;
+    s_u8[(size_t)n * G + 2 * kb + 1] = (prm >> 16) & 0xFF;
+    a[(size_t)n * G + 2 * kb + 1] = prm >> 24;
+  } else {
+    s_u8[(size_t)n * G + kb] = prm & 0xFF;
+    a[(size_t)n * G + kb] = (prm >> 8) & 0xFF;
+  }
+  if (kb == 0)
+    s_w_out[n] = reinterpret_cast<const float*>(packed + sw_offset_bytes())[n];
+  uint8_t* out = codes + (size_t)n * K + (size_t)kb * kTileK;
+  for (int c = 0; c < 4; ++c) {
+    uint4 v = *reinterpret_cast<const uint4*>(src + (c * kTileN + r) * 16);
+    uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    for (int j = 0; j < 4; ++j)
+      for (int b = 0; b < 4; ++b) {
+        uint32_t byte = (w4[j] >> (8 * b)) & 0xFF;
+        out[32 * c + 8 * j + b] = byte & 0xF;
+        out[32 * c + 8 * j + 4 + b] = byte >> 4;
+      }
+  }
+}
+
+// Per-token activation quantization: one CTA per token row.  Pass 1 finds
+// the row's absmax, pass 2 (re-reading the row, now in L1/L2) writes the
+// INT8 codes four at a time.
+constexpr int kActThreads = 256;
+
+__global__ void __launch_bounds__(kActThreads) act_quant_kernel(
+    const float* __restrict__ X, int M, int K, int8_t* __restrict__ Xq,
+    float* __restrict__ s_x) {
+  __shared__ float red[kActThreads / 32];
+  const int m = blockIdx.x;
+  const float4* row = reinterpret_cast<const float4*>(X + (size_t)m * K);
+  const int n4 = K / 4;
+  float amax = 0.0f;
+  for (int i = threadIdx.x; i < n4; i += kActThreads) {
+    float4 v = __ldg(row + i);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)),
+                             fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < kActThreads / 32 ? red[threadIdx.x] : 0.0f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float s = __fdiv_rn(red[0], 127.0f);
+  if (threadIdx.x == 0) s_x[m] = s;
+  uint32_t* out = reinterpret_cast<uint32_t*>(Xq + (size_t)m * K);
+  for (int i = threadIdx.x; i < n4; i += kActThreads) {
+    float4 v = __ldg(row + i);
+    uint32_t q = (uint32_t)(quant_sym(v.x, s, 127) & 0xFF) |
+                 ((uint32_t)(quant_sym(v.y, s, 127) & 0xFF) << 8) |
+                 ((uint32_t)(quant_sym(v.z, s, 127) & 0xFF) << 16) |
+                 ((uint32_t)(quant_sym(v.w, s, 127) & 0xFF) << 24);
+    out[i] = q;
+  }
+}
+
+}  // namespace w4a8

@@ -1,0 +1,330 @@
+// w4a8_api.cu -- the C ABI of libw4a8.so (declared in include/w4a8.h):
+// host-side argument checks, schedule selection, tensor-map encoding and
+// kernel launches.  One translation unit: the kernels live in the .cuh
+// files included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gemm.cuh"
+#include "layout.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+#include "w4a8.h"
+
+namespace w4a8 {
+
+
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr int kMaxDevices = 64;
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+
+int num_sms(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map over Xq [M][K] int8 (K contiguous): boxes of 128 bytes of k by
+// `rows` tokens, 128-byte swizzle, zero fill past row M.
+bool make_act_map(CUtensorMap* map, const int8_t* Xq, int M, int K, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(Xq), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ schedule
+struct Schedule {
+  int T = 16, splits = 1, kt_per = 1, n_tiles = 1, m_tiles = 1, ctas = 1;
+};
+
+int ctas_per_sm(int T) { return T <= 128 ? 2 : 1; }
+
+Schedule choose_schedule(int M, int N, int K, int sms) {
+  Schedule s;
+  s.T = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  s.n_tiles = (N + kTileN - 1) / kTileN;
+  s.m_tiles = M > 0 ? (M + s.T - 1) / s.T : 0;
+  const int kt = K / kTileK;
+  const int tiles = s.n_tiles * s.m_tiles;
+  int splits = 1;
+  if (tiles > 0 && tiles < sms) {
+    splits = (sms * ctas_per_sm(s.T)) / tiles;
+    if (splits < 1) splits = 1;
+    if (splits > kt) splits = kt;
+  }
+  s.kt_per = (kt + splits - 1) / splits;
+  s.splits = (kt + s.kt_per - 1) / s.kt_per;  // no empty split
+  s.ctas = tiles * s.splits;
+  return s;
+}
+
+size_t workspace_bytes_for(const Schedule& s, int N) {
+  if (s.splits <= 1) return 0;
+  const size_t n_pad = (size_t)round_up(N, kTileN);
+  size_t partial = (size_t)s.m_tiles * n_pad * s.T * sizeof(int32_t);
+  partial = (partial + 255) / 256 * 256;
+  return partial + (size_t)s.m_tiles * s.n_tiles * sizeof(uint32_t);
+}
+
+// ------------------------------------------------------------- launches
+template <int T, int STAGES, int DQG, int MINB>
+cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
+                        cudaStream_t st) {
+  using C = GemmCfg<T, STAGES, DQG>;
+  auto k = w4a8_gemm_kernel<T, STAGES, DQG, MINB>;
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_relaxed);
+  }
+  k<<<ctas, C::kThreads, C::kSmemBytes, st>>>(map, p);
+  return cudaGetLastError();
+}
+
+int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
+                int K, uint16_t* Y, int32_t* acc, void* workspace, size_t ws_bytes,
+                void* stream) {
+  if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return W4A8_OK;
+  if (!Xq || !packed || (!Y && !acc) || (Y && !s_x)) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(packed, 16) || (Y && !aligned(Y, 2)) ||
+      (acc && !aligned(acc, 4)) || (s_x && !aligned(s_x, 4)))
+    return W4A8_ERR_MISALIGNED;
+  const int dev = current_device();
+  if (dev < 0) return W4A8_ERR_CUDA;
+  const Schedule s = choose_schedule(M, N, K, num_sms(dev));
+  const size_t need = workspace_bytes_for(s, N);
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
+    return W4A8_ERR_WORKSPACE;
+
+  const int n_pad = round_up(N, kTileN);
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  GemmParams p;
+  p.tiles = base + tiles_offset_bytes(n_pad);
+  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
+  p.s_x = s_x;
+  p.Y = Y;
+  p.acc = Y ? nullptr : acc;
+  p.ws = static_cast<int32_t*>(workspace);
+  size_t partial = need ? ((size_t)s.m_tiles * n_pad * s.T * 4 + 255) / 256 * 256 : 0;
+  p.counters = need ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + partial)
+                    : nullptr;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_pad = n_pad;
+  p.kt_total = K / kTileK;
+  p.splits = s.splits;
+  p.kt_per_split = s.kt_per;
+  p.n_tiles = s.n_tiles;
+  p.m_tiles = s.m_tiles;
+  p.wait_limit_ns = kWaitLimitNs;
+  p.hdr = reinterpret_cast<const PackedHeader*>(base);
+
+  CUtensorMap map;
+  if (!make_act_map(&map, Xq, M, K, s.T)) return W4A8_ERR_CUDA;
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e;
+  switch (s.T) {
+    case 16: e = launch_gemm<16, 6, 2, 2>(map, p, s.ctas, st); break;
+    case 32: e = launch_gemm<32, 6, 2, 2>(map, p, s.ctas, st); break;
+    case 64: e = launch_gemm<64, 6, 2, 2>(map, p, s.ctas, st); break;
+    case 128: e = launch_gemm<128, 4, 2, 2>(map, p, s.ctas, st); break;
+    default: e = launch_gemm<256, 5, 2, 1>(map, p, s.ctas, st); break;
+  }
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+__global__ void timeout_probe_kernel(unsigned long long limit_ns) {
+  __shared__ alignas(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on this barrier: the bounded wait must give up
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, nullptr, limit_ns);
+}
+
+}  // namespace
+}  // namespace w4a8
+
+using namespace w4a8;
+
+extern "C" {
+
+const char* w4a8_status_string(int status) {
+  switch (status) {
+    case W4A8_OK: return "W4A8_OK";
+    case W4A8_ERR_INVALID_ARG: return "W4A8_ERR_INVALID_ARG";
+    case W4A8_ERR_UNSUPPORTED_SHAPE: return "W4A8_ERR_UNSUPPORTED_SHAPE";
+    case W4A8_ERR_MISALIGNED: return "W4A8_ERR_MISALIGNED";
+    case W4A8_ERR_WORKSPACE: return "W4A8_ERR_WORKSPACE";
+    case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
+    case W4A8_ERR_TIMEOUT: return "W4A8_ERR_TIMEOUT";
+    case W4A8_ERR_BAD_PACKED: return "W4A8_ERR_BAD_PACKED";
+    default: return "W4A8_ERR_UNKNOWN";
+  }
+}
+
+int w4a8_version(void) { return 1; }
+
+size_t w4a8_packed_weight_bytes(int N, int K, int group) {
+  if (N < 1 || K < 1 || K % kTileK != 0 || K > 65536 || (group != 64 && group != 128))
+    return 0;
+  return (size_t)packed_bytes(N, K);
+}
+
+int w4a8_quantize_weights(const float* W, int N, int K, int group, void* packed,
+                          void* stream) {
+  if (!W || !packed || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (group != 64 && group != 128) return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(W, 16) || !aligned(packed, 16)) return W4A8_ERR_MISALIGNED;
+  const int dev = current_device();
+  if (dev < 0) return W4A8_ERR_CUDA;
+  const int n_pad = round_up(N, kTileN);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* out = static_cast<uint8_t*>(packed);
+  weight_scale_kernel<<<(n_pad + 7) / 8, 256, 0, st>>>(W, N, K, group, n_pad, out);
+  if (cudaGetLastError() != cudaSuccess) return W4A8_ERR_CUDA;
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if (dev < kMaxDevices && !attr_set[dev].load()) {
+    if (cudaFuncSetAttribute(weight_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPackSmemBytes) != cudaSuccess)
+      return W4A8_ERR_CUDA;
+    attr_set[dev].store(true);
+  }
+  dim3 grid(K / kTileK, n_pad / kTileN);
+  weight_pack_kernel<<<grid, 128, kPackSmemBytes, st>>>(W, N, K, group, n_pad, out);
+  return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+int w4a8_unpack_weights(const void* packed, int N, int K, uint8_t* codes, uint8_t* s_u8,
+                        uint8_t* a, float* s_w, void* stream) {
+  if (!packed || !codes || !s_u8 || !a || !s_w || N < 1 || K < 1)
+    return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(packed, 16) || !aligned(s_w, 4)) return W4A8_ERR_MISALIGNED;
+  const int n_pad = round_up(N, kTileN);
+  dim3 grid(K / kTileK, n_pad / kTileN);
+  weight_unpack_kernel<<<grid, 128, 0, as_stream(stream)>>>(
+      static_cast<const uint8_t*>(packed), N, K, n_pad, codes, s_u8, a, s_w);
+  return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+int w4a8_quantize_act(const float* X, int M, int K, int8_t* Xq, float* s_x, void* stream) {
+  if (M < 0 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return W4A8_OK;
+  if (!X || !Xq || !s_x) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(s_x, 4)) return W4A8_ERR_MISALIGNED;
+  act_quant_kernel<<<M, kActThreads, 0, as_stream(stream)>>>(X, M, K, Xq, s_x);
+  return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+size_t w4a8_gemm_workspace_bytes(int M, int N, int K) {
+  if (M < 1 || N < 1 || K < 1 || K % kTileK != 0) return 0;
+  const int dev = current_device();
+  return workspace_bytes_for(choose_schedule(M, N, K, num_sms(dev < 0 ? 0 : dev)), N);
+}
+
+int w4a8_workspace_init(void* workspace, size_t bytes, void* stream) {
+  if (bytes == 0) return W4A8_OK;
+  if (!workspace) return W4A8_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, bytes, as_stream(stream)) == cudaSuccess
+             ? W4A8_OK
+             : W4A8_ERR_CUDA;
+}
+
+int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M, int N, int K,
+              uint16_t* Y, void* workspace, size_t ws_bytes, void* stream) {
+  if (M > 0 && !Y) return W4A8_ERR_INVALID_ARG;
+  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, workspace, ws_bytes, stream);
+}
+
+int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K, int32_t* acc,
+                  void* workspace, size_t ws_bytes, void* stream) {
+  if (M > 0 && !acc) return W4A8_ERR_INVALID_ARG;
+  return gemm_common(Xq, nullptr, packed, M, N, K, nullptr, acc, workspace, ws_bytes,
+                     stream);
+}
+
+int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits, int* ctas) {
+  if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const Schedule s = choose_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev));
+  if (tile_tokens) *tile_tokens = s.T;
+  if (splits) *splits = s.splits;
+  if (ctas) *ctas = s.ctas;
+  return W4A8_OK;
+}
+
+int w4a8_get_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return W4A8_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return W4A8_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return W4A8_ERR_CUDA;
+  return v;
+}
+
+int w4a8_debug_timeout_probe(long long limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return W4A8_ERR_INVALID_ARG;
+  timeout_probe_kernel<<<1, 32, 0, as_stream(stream)>>>((unsigned long long)limit_ns);
+  return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+}  // extern "C"

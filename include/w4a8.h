@@ -1,0 +1,180 @@
+/*
+ * w4a8.h -- C ABI of libw4a8.so, a block-quantized W4A8 GEMM for NVIDIA
+ * B200 (sm_100a) in the style of LiquidGEMM / LiquidQuant (LQQ).
+ *
+ * The method (review page "LiquidGEMM", pith.science verdict on arXiv
+ * 2509.01229; field names of that page and the paper sections they quote):
+ *   - weights: per-output-channel symmetric INT8 in the protective range
+ *     [-119, 119] with an FP scale s_w (referee major 3, paper Sec. 4 Eq. 7),
+ *     then per group of 64 along K (skeptic concrete_test) shifted by the
+ *     group minimum into UINT8 and quantized to UINT4 codes with an integer
+ *     scale s_u8 <= 16 and an offset a = 2^7 + min (referee summary;
+ *     key_machinery; referee minor 2, Sec. 4 Eq. 10);
+ *   - dequantization inside the GEMM: (q_u4 * s_u8 + a) XOR 0x80, integer
+ *     multiply-add and a bit flip that never leave UINT8 (key_machinery;
+ *     referee summary; desk_editor);
+ *   - activations: per-token INT8 with an FP scale (supporting citation [29]);
+ *   - INT8 x INT8 tensor-core products accumulated in INT32 (lead), followed
+ *     by an FP epilogue y = s_x[m] * s_w[n] * acc[m][n] stored as bf16.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named X, W, Xq, s_x, packed, Y, acc, workspace and the outputs
+ *     of the unpack call are DEVICE pointers owned by the caller.  The library
+ *     allocates no memory and never synchronizes the host, except in
+ *     w4a8_get_status.  Work is enqueued on `stream` (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream) in call order.
+ *   - Matrices are row-major with the last index contiguous:
+ *       W  float32 [N][K]  (output channel n, reduction index k)
+ *       X  float32 [M][K]  (token m)
+ *       Xq int8    [M][K],  s_x float32 [M]
+ *       Y  bf16    [M][N]   (stored as uint16 bit patterns)
+ *       acc int32  [M][N]
+ *   - Supported shapes: M >= 0, N >= 1, K a positive multiple of 128,
+ *     K <= 65536, group = 64 or 128.  M == 0 is a no-op.  Other shapes return
+ *     W4A8_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ *   - Alignment: Xq, X, W and the packed buffer must be 16-byte aligned,
+ *     Y and acc 4-byte aligned; otherwise W4A8_ERR_MISALIGNED.
+ *   - Return value: W4A8_OK or a negative w4a8_status.  Argument errors are
+ *     detected on the host before any launch.  A launch failure returns
+ *     W4A8_ERR_CUDA.  Errors found on the device (a bounded wait that ran out)
+ *     are recorded in a per-device status word read by w4a8_get_status.
+ *   - Inputs must be finite; NaN or Inf inputs give unspecified codes.
+ */
+#ifndef W4A8_H
+#define W4A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  W4A8_OK = 0,
+  W4A8_ERR_INVALID_ARG = -1,       /* NULL pointer, negative size, bad group */
+  W4A8_ERR_UNSUPPORTED_SHAPE = -2, /* K % 128, K > 65536, N < 1 */
+  W4A8_ERR_MISALIGNED = -3,        /* see the alignment rule above */
+  W4A8_ERR_WORKSPACE = -4,         /* workspace NULL or smaller than required */
+  W4A8_ERR_CUDA = -5,              /* a CUDA runtime call failed */
+  W4A8_ERR_TIMEOUT = -6,           /* a device-side bounded wait ran out */
+  W4A8_ERR_BAD_PACKED = -7         /* packed buffer header does not match */
+} w4a8_status;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* w4a8_status_string(int status);
+
+/* Library ABI version (currently 1). */
+int w4a8_version(void);
+
+/*
+ * Size in bytes of the packed LQQ weight buffer for an N x K layer.
+ * Layout (all offsets from the buffer start):
+ *   [0, 256)       header: magic 'W4A8', version, N, K, group, padded N
+ *   [256, ...)     s_w: float32 per output channel, N rounded up to 128
+ *   tiles          one 8704-byte tile per (128 output channels, 128 k):
+ *                  8192 bytes of 4-bit codes then 512 bytes of (s_u8, a)
+ *                  pairs, tiles ordered by output-channel block, then k.
+ * Returns 0 for an unsupported shape.  Host-only, no CUDA call.
+ */
+size_t w4a8_packed_weight_bytes(int N, int K, int group);
+
+/*
+ * Offline weight quantization and packing (review: key_machinery; referee
+ * summary; referee major 3 and minor 2, paper Sec. 4 Eqs. 7 and 10).
+ *   W       [N][K] float32, device
+ *   packed  device buffer of w4a8_packed_weight_bytes(N, K, group) bytes,
+ *           fully written by this call (padding included)
+ * Level 1: s_w[n] = max_k |W[n][k]| / 119 (fp32 division);
+ *          Q = clamp(rint(W / s_w), -119, 119), ties to even; s_w = 0 gives 0.
+ * Level 2, per group of `group` k-values in one row: mn/mx = min/max of Q,
+ *          s_u8 = max(1, ceil((mx - mn) / 15)), a = 128 + mn,
+ *          code = floor((2 (Q - mn) + s_u8) / (2 s_u8)) in [0, 15].
+ */
+int w4a8_quantize_weights(const float* W, int N, int K, int group,
+                          void* packed, void* stream);
+
+/*
+ * Test aid: expand a packed buffer back into canonical arrays.
+ *   codes [N][K] uint8 (one code per byte), s_u8 [N][K/group] uint8,
+ *   a [N][K/group] uint8, s_w [N] float32.  All device pointers.
+ * N, K and group are read from the header; pass the same N and K as a check.
+ */
+int w4a8_unpack_weights(const void* packed, int N, int K, uint8_t* codes,
+                        uint8_t* s_u8, uint8_t* a, float* s_w, void* stream);
+
+/*
+ * Per-token activation quantization (supporting citation [29]; symmetric
+ * range +-127):  s_x[m] = max_k |X[m][k]| / 127 (fp32 division),
+ * Xq[m][k] = clamp(rint(X[m][k] / s_x[m]), -127, 127), ties to even;
+ * an all-zero row gives s_x = 0 and Xq = 0.
+ *   X [M][K] float32 -> Xq [M][K] int8, s_x [M] float32 (device).
+ * K only needs to be a positive multiple of 16 here.
+ */
+int w4a8_quantize_act(const float* X, int M, int K, int8_t* Xq, float* s_x,
+                      void* stream);
+
+/*
+ * Bytes of device workspace w4a8_gemm / w4a8_gemm_i32 need for this shape
+ * (0 when the chosen schedule needs none).  The workspace holds INT32
+ * split-K partial sums and arrival counters.  It must be zero-filled before
+ * its first use (cudaMemset, or w4a8_workspace_init); every successful call
+ * leaves it zero-filled again, so it can be reused by later calls on the
+ * same stream without clearing.  After a call that reported an error,
+ * initialize it again.  Two calls that may run at the same time on the GPU
+ * must not share a workspace.
+ */
+size_t w4a8_gemm_workspace_bytes(int M, int N, int K);
+
+/* Zero-fill a workspace of `bytes` bytes on `stream`. */
+int w4a8_workspace_init(void* workspace, size_t bytes, void* stream);
+
+/*
+ * The W4A8 GEMM with the fused bf16 epilogue:
+ *   Y[m][n] = bf16_rn( float(acc[m][n]) * (s_x[m] * s_w[n]) ),
+ *   acc[m][n] = sum_k Xq[m][k] * (code[n][k] * s_u8 + a - 128)   (INT32)
+ * with the weights dequantized in-kernel as (code * s_u8 + a) XOR 0x80
+ * (key_machinery) and the products on tcgen05 INT8 tensor cores (lead).
+ *   Xq [M][K] int8, s_x [M] float32, packed (from w4a8_quantize_weights),
+ *   Y [M][N] bf16, workspace of w4a8_gemm_workspace_bytes(M, N, K) bytes.
+ * The accumulator is exact; the epilogue differs from an exact FP64
+ * evaluation by at most one bf16 ulp.
+ */
+int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M,
+              int N, int K, uint16_t* Y, void* workspace, size_t ws_bytes,
+              void* stream);
+
+/* Same product, writing the exact INT32 accumulators acc [M][N] instead of
+ * the bf16 output (for bit-exact verification). */
+int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K,
+                  int32_t* acc, void* workspace, size_t ws_bytes,
+                  void* stream);
+
+/*
+ * Schedule the library picks for a shape (introspection for tests and
+ * benchmarks): tokens per tile, split-K factor, number of CTAs.  Any output
+ * pointer may be NULL.  Host-only.
+ */
+int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
+                       int* ctas);
+
+/*
+ * Waits for `stream`, then returns and clears the device status word of the
+ * current device: W4A8_OK, or W4A8_ERR_TIMEOUT if a kernel's bounded wait
+ * ran out since the last call.  W4A8_ERR_CUDA if the synchronization failed.
+ */
+int w4a8_get_status(void* stream);
+
+/*
+ * Test aid for the failure path: launches one CTA that waits on a shared
+ * memory barrier nothing ever arrives on, with a wait limit of `limit_ns`
+ * nanoseconds (1e3 .. 1e10).  The kernel records W4A8_ERR_TIMEOUT in the
+ * status word and returns; nothing faults or hangs.
+ */
+int w4a8_debug_timeout_probe(long long limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A8_H */
