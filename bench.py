@@ -1,0 +1,529 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 W4A8 GEMM path on the decode-sweep workload.
+
+One step = the per-call hot path for every M of the sweep N = K = 4096,
+M in {1, 2, 4, 8, 16, 32, 64, 128, 256}: per-token activation quantization
+of fp32 X [M, K] followed by the W4A8 GEMM with the bf16 epilogue.  The
+weights are packed once, offline (LQQ weight quantization and packing are
+timed separately and reported as ``offline_pack``).
+
+* value: weight GB/s over the whole step (packed weight bytes of the nine
+  GEMMs / step time), device time with CUDA events, max over ranks, one CUDA
+  graph per step, 32 rotating copies of the packed weights (285 MB, more than
+  twice the L2) so every GEMM streams its weights from HBM.
+* roofline: the GEMM kernel, algorithmic bytes per launch / its average
+  launch duration (CUDA events around graphs of back-to-back launches on the
+  launching stream), against the measured HBM copy bandwidth; per-M figures
+  with the bound that applies (HBM or INT8 tensor) are in ``sweep``.
+* e2e: the same metric through the public calls with host buffers: each
+  step copies X from pinned host memory, quantizes, multiplies and copies Y
+  back, eagerly (no graph).
+* cpu_baseline: the CPU oracle timed on a bounded sample of the same
+  workload on the host cores (rank 0, one GPU only).
+
+``--impl reference`` times the CPU oracle alone as the reference arm.
+Multi-GPU (torchrun): independent replicas, one per GPU, no collective on
+the data path; the step time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_block_quantized_w4a8_b200 import workloads as wl  # noqa: E402
+
+WORKLOAD = "decode_sweep_4096"
+METRIC = "W4A8 GEMM TOPS & weight GB/s vs M (1 B200), as % of INT8/HBM roofline"
+UNIT = "GB/s"
+N_COPIES = 32
+GROUP = 64
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense INT8 / bf16 tensor throughput on B200
+
+
+# ------------------------------------------------------------------ units
+def weight_bytes(N, K):
+    """Packed LQQ weight bytes a GEMM must read: codes + (s_u8, a) + s_w."""
+    return N * K // 2 + 2 * N * (K // GROUP) + 4 * N
+
+
+def gemm_bytes(M, N, K):
+    """Algorithmic HBM bytes of one GEMM: weights + Xq + s_x + Y (bf16)."""
+    return weight_bytes(N, K) + M * K + 4 * M + 2 * M * N
+
+
+def gemm_ops(M, N, K):
+    return 2 * M * N * K
+
+
+def act_bytes(M, K):
+    """Activation quantization: read fp32 X, write int8 Xq and s_x."""
+    return 5 * M * K + 4 * M
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS,
+                    bf16_sust=1400.0, source="fallback")
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "bit_block_quantized_w4a8_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("csrc_digest") != csrc_digest():
+        return None
+    return d
+
+
+# ------------------------------------------------------------ distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_init(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world > 1
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(units_per_rank, world, elapsed_max_s):
+    """Whole-job throughput of independent replicas: all ranks' units over
+    the slowest rank's time."""
+    return units_per_rank * world / elapsed_max_s
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(p[1]), smax=float(p[2]), reasons=p[4:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        active = sorted({names[i] for r in rows for i in range(4)
+                         if r["reasons"][i + 1].lower().startswith("active")})
+        loaded = [r["sm"] for r in rows if r["sm"] > 0.5 * r["smax"]] or [r["sm"] for r in rows]
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": rows[0]["smax"],
+                "reasons": active, "samples": len(rows)}
+
+
+# ------------------------------------------------------- oracle (CPU) arm
+def _oracle_inputs(Ms):
+    import oracle
+    layer = wl.WORKLOADS[WORKLOAD].layers[0]
+    W = wl.layer_weights(WORKLOAD, layer).numpy()
+    wq = oracle.quantize_weights(W, group=GROUP)
+    xs = {M: wl.layer_activations(WORKLOAD, layer, M).numpy() for M in Ms}
+    return wq, xs
+
+
+def _rows(wq, n):
+    return {k: np.ascontiguousarray(v[:n]) for k, v in wq.items()}
+
+
+def _oracle_call(x, wq):
+    """One oracle pass of the per-call path: activation quantization, then
+    dequantization, integer GEMM and FP64 epilogue."""
+    import oracle
+    Xq, sx = oracle.quantize_act(x)
+    oracle.w4a8_gemm(Xq, sx, wq, group=GROUP, want_acc=False)
+
+
+def cpu_baseline(N, K, Ms, budget_s=20.0):
+    """Oracle throughput in the bench's unit on a bounded sample: the sweep's
+    Ms in increasing order, each once, until the CPU budget is spent."""
+    import oracle
+    wq, xs = _oracle_inputs(Ms)
+    done, t = [], 0.0
+    for M in Ms:
+        t0 = time.perf_counter()
+        _oracle_call(xs[M], wq)
+        t += time.perf_counter() - t0
+        done.append(M)
+        if t > budget_s:
+            break
+    value = len(done) * weight_bytes(N, K) / t / 1e9
+    return {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "one oracle pass per M in %s (N=K=%d): activation quantization, "
+                      "dequantization, integer GEMM, FP64 epilogue" % (done, K),
+            "seconds": t}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is one M=1 decode call on a
+    slice of the layer's output channels, the slice sized so that warm-up and
+    timed steps together stay within about two and a half minutes."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    layer = wl.WORKLOADS[WORKLOAD].layers[0]
+    N, K = layer.N, layer.K
+    wq, xs = _oracle_inputs([1])
+    t0 = time.perf_counter()
+    _oracle_call(xs[1], wq)
+    t_full = time.perf_counter() - t0
+    per_step = 150.0 / (args.steps + args.warmup)
+    n_sub = int(N * per_step / max(t_full, 1e-9)) // 128 * 128
+    n_sub = max(128, min(N, n_sub))
+    ws = _rows(wq, n_sub)
+    for _ in range(args.warmup):
+        _oracle_call(xs[1], ws)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_call(xs[1], ws)
+    t = (time.perf_counter() - t0) / args.steps
+    value = weight_bytes(n_sub, K) / t / 1e9
+    sample = ("per step: one M=1 call on output channels [0, %d) of the N=K=%d layer "
+              "(activation quantization, dequantization, integer GEMM, FP64 epilogue)"
+              % (n_sub, K))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "N": N, "K": K, "Ms": list(wl.WORKLOADS[WORKLOAD].Ms),
+                   "note": "CPU oracle on a bounded sample of the workload"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- CUDA arm
+def _graph(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def _time_graph(g, reps, stream):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / reps
+
+
+def run_cuda(args):
+    import bit_block_quantized_w4a8_b200 as w4
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    peaks = load_peaks()
+    layer = wl.WORKLOADS[WORKLOAD].layers[0]
+    N, K = layer.N, layer.K
+    Ms = list(wl.WORKLOADS[WORKLOAD].Ms)
+
+    # ---- offline: quantize + pack the layer once, then rotating copies
+    W = wl.layer_weights(WORKLOAD, layer).to(dev)
+    w4.w4a8_quantize_weights(W)  # warm-up of the packer
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    pk0 = w4.w4a8_quantize_weights(W)
+    e1.record()
+    e1.synchronize()
+    pack_s = e0.elapsed_time(e1) / 1e3
+    copies = [pk0] + [w4.PackedWeights(pk0.data.clone(), N, K, GROUP) for _ in range(N_COPIES - 1)]
+    del W
+
+    Xs = {M: wl.layer_activations(WORKLOAD, layer, M).to(dev) for M in Ms}
+    Xq = {M: torch.empty(M, K, dtype=torch.int8, device=dev) for M in Ms}
+    sx = {M: torch.empty(M, dtype=torch.float32, device=dev) for M in Ms}
+    Ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in Ms}
+    ws_need = max(w4.w4a8_gemm_workspace_bytes(M, N, K) for M in Ms)
+    ws = torch.zeros(max(ws_need, 256), dtype=torch.uint8, device=dev)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step_fn(r):
+        def fn():
+            for j, M in enumerate(Ms):
+                w4.w4a8_quantize_act(Xs[M], out=Xq[M], scale_out=sx[M], stream=stream)
+                w4.w4a8_gemm(Xq[M], sx[M], copies[(r * len(Ms) + j) % N_COPIES], out=Ys[M],
+                             workspace=ws, stream=stream)
+        return fn
+
+    with torch.cuda.stream(stream):
+        for r in range(2):  # eager warm-up: kernel attributes, tensor-map entry point
+            step_fn(r)()
+    stream.synchronize()
+    assert w4.w4a8_get_status(stream) == 0
+    n_graphs = N_COPIES
+    graphs = [_graph(step_fn(r), stream) for r in range(n_graphs)]
+
+    for s in range(args.warmup):
+        graphs[s % n_graphs].replay()
+    stream.synchronize()
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        graphs[s % n_graphs].replay()
+    t1.record(stream)
+    t1.synchronize()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(world, dev)
+    elapsed = t0.elapsed_time(t1) / 1e3
+    elapsed_max = max_over_ranks(elapsed, world, dev)
+    status = w4.w4a8_get_status(stream)
+    if status != 0:
+        raise RuntimeError("device status after the timed region: %s" % w4.w4a8_status_string(status))
+
+    wbytes_step = len(Ms) * weight_bytes(N, K)
+    value = replica_value(wbytes_step * args.steps, world, elapsed_max) / 1e9
+    ops_step = sum(gemm_ops(M, N, K) for M in Ms)
+    tops = ops_step * args.steps * world / elapsed_max / 1e12
+
+    # ---- per-kernel durations: graphs of back-to-back launches of one kernel
+    per_m = []
+    reps = 10
+    for M in Ms:
+        def gemms(M=M):
+            for i in range(N_COPIES):
+                w4.w4a8_gemm(Xq[M], sx[M], copies[i], out=Ys[M], workspace=ws, stream=stream)
+
+        def quants(M=M):
+            for i in range(N_COPIES):
+                w4.w4a8_quantize_act(Xs[M], out=Xq[M], scale_out=sx[M], stream=stream)
+        gg, gq = _graph(gemms, stream), _graph(quants, stream)
+        gg.replay()
+        gq.replay()
+        tg = _time_graph(gg, reps, stream) / N_COPIES
+        tq = _time_graph(gq, reps, stream) / N_COPIES
+        b, o = gemm_bytes(M, N, K), gemm_ops(M, N, K)
+        hbm_t, tc_t = b / (peaks["hbm"] * 1e9), o / (peaks["bf16"] * INT8_PER_BF16 * 1e12)
+        bound = "hbm" if hbm_t >= tc_t else "tensor"
+        frac = (hbm_t if bound == "hbm" else tc_t) / tg
+        T, splits, ctas = w4.w4a8_gemm_schedule(M, N, K)
+        per_m.append({"M": M, "gemm_us": tg * 1e6, "act_quant_us": tq * 1e6,
+                      "tops": o / tg / 1e12, "weight_gbs": weight_bytes(N, K) / tg / 1e9,
+                      "total_gbs": b / tg / 1e9, "bound": bound, "frac": frac,
+                      "act_quant_gbs": act_bytes(M, K) / tq / 1e9,
+                      "schedule": {"tile_tokens": T, "splits": splits, "ctas": ctas}})
+        del gg, gq
+    stream.synchronize()
+    bytes_all = sum(gemm_bytes(M, N, K) for M in Ms)
+    dur_all = sum(r["gemm_us"] for r in per_m) * 1e-6
+    achieved = bytes_all / dur_all / 1e9
+    prof = profiled_traffic()
+    traffic = None
+    if prof is not None:
+        traffic = prof.get("sweep_mean_dram_bytes_per_launch")
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm"], "traffic": traffic,
+                "kernel": "w4a8_gemm_kernel", "peak_source": peaks["source"],
+                "note": "algorithmic bytes of the nine sweep launches / their summed average "
+                        "launch durations"}
+
+    # ---- e2e: public calls with host buffers, copies inside the timed region
+    e2e_steps = max(1, min(args.steps, 200))
+    hX = {M: Xs[M].cpu().pin_memory() for M in Ms}
+    hY = {M: torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in Ms}
+    dX = {M: torch.empty_like(Xs[M]) for M in Ms}
+
+    def e2e_step(r):
+        for j, M in enumerate(Ms):
+            dX[M].copy_(hX[M], non_blocking=True)
+            xq, s_ = w4.w4a8_quantize_act(dX[M], out=Xq[M], scale_out=sx[M], stream=stream)
+            y = w4.w4a8_gemm(xq, s_, copies[(r * len(Ms) + j) % N_COPIES], out=Ys[M],
+                             workspace=ws, stream=stream)
+            hY[M].copy_(y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for r in range(3):
+            e2e_step(r)
+        stream.synchronize()
+        barrier(world, dev)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for r in range(e2e_steps):
+            e2e_step(r)
+        a1.record(stream)
+    a1.synchronize()
+    e2e_el = max_over_ranks(a0.elapsed_time(a1) / 1e3, world, dev)
+    e2e_value = replica_value(wbytes_step * e2e_steps, world, e2e_el) / 1e9
+    h2d = sum(M * K * 4 for M in Ms)
+    d2h = sum(M * N * 2 for M in Ms)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(N, K, Ms, budget_s=args.cpu_budget)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed_max / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "N": N, "K": K, "Ms": Ms, "group": GROUP,
+                   "step": "per M: activation quantization + W4A8 GEMM (bf16 epilogue)",
+                   "l2": "inputs larger than L2: %d rotating packed weight copies (%.0f MB)"
+                         % (N_COPIES, N_COPIES * w4.w4a8_packed_weight_bytes(N, K) / 1e6),
+                   "launch": "one CUDA graph per step", "parallelism": "replicas"},
+        "tops": tops,
+        "gpu_launches": 2 * len(Ms) * args.steps,
+        "roofline": roofline,
+        "sweep": per_m,
+        "offline_pack": {"seconds": pack_s, "fp32_weight_gbs": 4 * N * K / pack_s / 1e9},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    graphs.clear()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_profile_case(args):
+    """Small fixed case for profilers: pack the N=K=4096 layer once and run
+    one GEMM per requested M (no graphs, no timing)."""
+    import bit_block_quantized_w4a8_b200 as w4
+    torch.cuda.set_device(0)
+    layer = wl.WORKLOADS[WORKLOAD].layers[0]
+    N, K = layer.N, layer.K
+    pk = w4.w4a8_quantize_weights(wl.layer_weights(WORKLOAD, layer).cuda())
+    for M in [int(x) for x in args.profile.split(",")]:
+        Xq, sx = w4.w4a8_quantize_act(wl.layer_activations(WORKLOAD, layer, M).cuda())
+        w4.w4a8_gemm(Xq, sx, pk)
+    torch.cuda.synchronize()
+    status = w4.w4a8_get_status()
+    print("profile case done, status %s" % w4.w4a8_status_string(status))
+    return 0 if status == 0 else 1
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of CPU work for the oracle baseline sample")
+    ap.add_argument("--profile", default=None,
+                    help="comma-separated Ms: run one GEMM each on N=K=4096 for a profiler")
+    args = ap.parse_args(argv)
+    if args.profile:
+        return run_profile_case(args)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cuda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -290,13 +290,11 @@ int w4a8_workspace_init(void* workspace, size_t bytes, void* stream) {
 
 int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M, int N, int K,
               uint16_t* Y, void* workspace, size_t ws_bytes, void* stream) {
-  if (M > 0 && !Y) return W4A8_ERR_INVALID_ARG;
   return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, workspace, ws_bytes, stream);
 }
 
 int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K, int32_t* acc,
                   void* workspace, size_t ws_bytes, void* stream) {
-  if (M > 0 && !acc) return W4A8_ERR_INVALID_ARG;
   return gemm_common(Xq, nullptr, packed, M, N, K, nullptr, acc, workspace, ws_bytes,
                      stream);
 }

@@ -1,0 +1,100 @@
+"""CPU-only checks of the boundary: the library builds for sm_100a, loads,
+exports every entry point include/w4a8.h declares, and its host-only
+functions (sizes, schedules, argument checks) behave as documented.  No
+kernel is launched."""
+import os
+import re
+import subprocess
+
+import pytest
+
+import bit_block_quantized_w4a8_b200 as w4
+from bit_block_quantized_w4a8_b200 import build as wbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a8.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    wbuild.build()
+    return w4.lib()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a8_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_three_calls():
+    names = _declared()
+    for n in ("w4a8_quantize_weights", "w4a8_quantize_act", "w4a8_gemm"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", wbuild.LIB]).decode()
+    exported = set(re.findall(r" T (w4a8_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        assert hasattr(L, n)
+
+
+def test_build_targets_sm100a_only():
+    flags = " ".join(wbuild.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert len(re.findall(r"arch=", flags)) == 1
+
+
+def test_packed_size(L):
+    # 4096 x 4096: header 256 + s_w 16 KiB + 32 x 32 tiles of 8704 bytes
+    assert w4.w4a8_packed_weight_bytes(4096, 4096) == 256 + 4 * 4096 + 32 * 32 * 8704
+    # ragged N is padded to 128 channels
+    n = w4.w4a8_packed_weight_bytes(200, 384)
+    assert n == 1280 + 2 * 3 * 8704
+    assert w4.w4a8_packed_weight_bytes(128, 200) == 0     # K % 128
+    assert w4.w4a8_packed_weight_bytes(128, 256, 32) == 0  # unsupported group
+    # about 0.531 bytes per weight
+    assert abs(w4.w4a8_packed_weight_bytes(28672, 8192) / (28672 * 8192) - 0.53125) < 1e-3
+
+
+def test_status_strings(L):
+    for code in range(-7, 1):
+        assert w4.w4a8_status_string(code).startswith("W4A8_")
+    assert w4.w4a8_status_string(-99) == "W4A8_ERR_UNKNOWN"
+    assert w4.w4a8_version() == 1
+
+
+def test_argument_checks_before_any_launch(L):
+    """Rejected calls return before touching the device."""
+    st = None
+    assert L.w4a8_gemm(None, None, None, 4, 128, 200, None, None, 0, st) == w4.ERR_UNSUPPORTED_SHAPE
+    assert L.w4a8_gemm(None, None, None, -1, 128, 256, None, None, 0, st) == w4.ERR_INVALID_ARG
+    assert L.w4a8_gemm(None, None, None, 0, 128, 256, None, None, 0, st) == w4.OK
+    assert L.w4a8_gemm_i32(None, None, 0, 128, 256, None, None, 0, st) == w4.OK
+    assert L.w4a8_gemm(None, None, None, 4, 128, 65536 + 128, None, None, 0, st) == w4.ERR_UNSUPPORTED_SHAPE
+    assert L.w4a8_quantize_act(None, 3, 100, None, None, st) == w4.ERR_UNSUPPORTED_SHAPE
+    assert L.w4a8_quantize_act(None, 0, 128, None, None, st) == w4.OK
+    assert L.w4a8_quantize_weights(None, 128, 256, 64, None, st) == w4.ERR_INVALID_ARG
+    assert L.w4a8_unpack_weights(None, 128, 256, None, None, None, None, st) == w4.ERR_INVALID_ARG
+    assert L.w4a8_debug_timeout_probe(10, st) == w4.ERR_INVALID_ARG
+
+
+def test_schedule_covers_the_machine(L):
+    # without a device the library assumes 148 SMs
+    T, splits, ctas = w4.w4a8_gemm_schedule(1, 4096, 4096)
+    assert T == 16 and splits > 1 and ctas <= 2 * 148 and ctas >= 148
+    T, splits, ctas = w4.w4a8_gemm_schedule(8192, 8192, 8192)
+    assert T == 256 and splits == 1 and ctas == 64 * 32
+    for M in (1, 2, 16, 17, 32, 33, 64, 65, 128, 129, 256, 257, 4096):
+        T, splits, ctas = w4.w4a8_gemm_schedule(M, 4096, 4096)
+        assert T >= min(M, 16) and T in (16, 32, 64, 128, 256)
+        assert 1 <= splits <= 32
+
+
+def test_workspace_sizes(L):
+    assert w4.w4a8_gemm_workspace_bytes(8192, 8192, 8192) == 0
+    ws = w4.w4a8_gemm_workspace_bytes(1, 4096, 4096)
+    assert ws >= 4096 * 16 * 4
