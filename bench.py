@@ -51,6 +51,7 @@ GROUP = 64
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0  # nominal dense INT8 / bf16 tensor throughput on B200
+PDL = 1  # W4A8_FLAG_PDL: consecutive calls overlap their weight fetch with the previous kernel
 
 
 # ------------------------------------------------------------------ units
@@ -298,10 +299,11 @@ def _graph(fn, stream):
 
 def _time_graph(g, reps, stream):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        g.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):  # replay() launches on the current stream
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
     e1.synchronize()
     return e0.elapsed_time(e1) / 1e3 / reps
 
@@ -343,9 +345,10 @@ def run_cuda(args):
     def step_fn(r):
         def fn():
             for j, M in enumerate(Ms):
-                w4.w4a8_quantize_act(Xs[M], out=Xq[M], scale_out=sx[M], stream=stream)
+                w4.w4a8_quantize_act(Xs[M], out=Xq[M], scale_out=sx[M], stream=stream,
+                                     flags=PDL)
                 w4.w4a8_gemm(Xq[M], sx[M], copies[(r * len(Ms) + j) % N_COPIES], out=Ys[M],
-                             workspace=ws, stream=stream)
+                             workspace=ws, stream=stream, flags=PDL)
         return fn
 
     with torch.cuda.stream(stream):
@@ -356,18 +359,20 @@ def run_cuda(args):
     n_graphs = N_COPIES
     graphs = [_graph(step_fn(r), stream) for r in range(n_graphs)]
 
-    for s in range(args.warmup):
-        graphs[s % n_graphs].replay()
+    with torch.cuda.stream(stream):  # replay() launches on the current stream
+        for s in range(args.warmup):
+            graphs[s % n_graphs].replay()
     stream.synchronize()
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     clocks = ClockSampler(local)
     clocks.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for s in range(args.steps):
-        graphs[s % n_graphs].replay()
-    t1.record(stream)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for s in range(args.steps):
+            graphs[s % n_graphs].replay()
+        t1.record(stream)
     t1.synchronize()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
@@ -387,29 +392,36 @@ def run_cuda(args):
     per_m = []
     reps = 10
     for M in Ms:
-        def gemms(M=M):
+        def gemms(M=M, fl=PDL):
             for i in range(N_COPIES):
-                w4.w4a8_gemm(Xq[M], sx[M], copies[i], out=Ys[M], workspace=ws, stream=stream)
+                w4.w4a8_gemm(Xq[M], sx[M], copies[i], out=Ys[M], workspace=ws, stream=stream,
+                             flags=fl)
 
         def quants(M=M):
             for i in range(N_COPIES):
-                w4.w4a8_quantize_act(Xs[M], out=Xq[M], scale_out=sx[M], stream=stream)
+                w4.w4a8_quantize_act(Xs[M], out=Xq[M], scale_out=sx[M], stream=stream,
+                                     flags=PDL)
         gg, gq = _graph(gemms, stream), _graph(quants, stream)
-        gg.replay()
-        gq.replay()
+        g0 = _graph(lambda M=M: gemms(M, 0), stream)
+        with torch.cuda.stream(stream):
+            gg.replay()
+            gq.replay()
+            g0.replay()
         tg = _time_graph(gg, reps, stream) / N_COPIES
         tq = _time_graph(gq, reps, stream) / N_COPIES
+        t_nopdl = _time_graph(g0, reps, stream) / N_COPIES
         b, o = gemm_bytes(M, N, K), gemm_ops(M, N, K)
         hbm_t, tc_t = b / (peaks["hbm"] * 1e9), o / (peaks["bf16"] * INT8_PER_BF16 * 1e12)
         bound = "hbm" if hbm_t >= tc_t else "tensor"
         frac = (hbm_t if bound == "hbm" else tc_t) / tg
         T, splits, ctas = w4.w4a8_gemm_schedule(M, N, K)
-        per_m.append({"M": M, "gemm_us": tg * 1e6, "act_quant_us": tq * 1e6,
+        per_m.append({"M": M, "gemm_us": tg * 1e6, "gemm_us_without_pdl": t_nopdl * 1e6,
+                      "act_quant_us": tq * 1e6,
                       "tops": o / tg / 1e12, "weight_gbs": weight_bytes(N, K) / tg / 1e9,
                       "total_gbs": b / tg / 1e9, "bound": bound, "frac": frac,
                       "act_quant_gbs": act_bytes(M, K) / tq / 1e9,
                       "schedule": {"tile_tokens": T, "splits": splits, "ctas": ctas}})
-        del gg, gq
+        del gg, gq, g0
     stream.synchronize()
     bytes_all = sum(gemm_bytes(M, N, K) for M in Ms)
     dur_all = sum(r["gemm_us"] for r in per_m) * 1e-6
@@ -433,9 +445,10 @@ def run_cuda(args):
     def e2e_step(r):
         for j, M in enumerate(Ms):
             dX[M].copy_(hX[M], non_blocking=True)
-            xq, s_ = w4.w4a8_quantize_act(dX[M], out=Xq[M], scale_out=sx[M], stream=stream)
+            xq, s_ = w4.w4a8_quantize_act(dX[M], out=Xq[M], scale_out=sx[M], stream=stream,
+                                          flags=PDL)
             y = w4.w4a8_gemm(xq, s_, copies[(r * len(Ms) + j) % N_COPIES], out=Ys[M],
-                             workspace=ws, stream=stream)
+                             workspace=ws, stream=stream, flags=PDL)
             hY[M].copy_(y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -467,7 +480,8 @@ def run_cuda(args):
                    "step": "per M: activation quantization + W4A8 GEMM (bf16 epilogue)",
                    "l2": "inputs larger than L2: %d rotating packed weight copies (%.0f MB)"
                          % (N_COPIES, N_COPIES * w4.w4a8_packed_weight_bytes(N, K) / 1e6),
-                   "launch": "one CUDA graph per step", "parallelism": "replicas"},
+                   "launch": "one CUDA graph per step, programmatic dependent launch",
+                   "parallelism": "replicas"},
         "tops": tops,
         "gpu_launches": 2 * len(Ms) * args.steps,
         "roofline": roofline,

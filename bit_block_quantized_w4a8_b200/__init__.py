@@ -36,6 +36,8 @@ ERR_CUDA = -5
 ERR_TIMEOUT = -6
 ERR_BAD_PACKED = -7
 
+W4A8_FLAG_PDL = 1  # programmatic dependent launch (see include/w4a8.h)
+
 
 class W4A8Error(RuntimeError):
     def __init__(self, what, code):
@@ -68,6 +70,8 @@ def lib():
             "w4a8_quantize_weights": ([p, i32, i32, i32, p, p], i32),
             "w4a8_unpack_weights": ([p, i32, i32, p, p, p, p, p], i32),
             "w4a8_quantize_act": ([p, i32, i32, p, p, p], i32),
+            "w4a8_quantize_act_ex": ([p, i32, i32, p, p, _ct.c_uint, p], i32),
+            "w4a8_gemm_ex": ([p, p, p, i32, i32, i32, p, p, sz, _ct.c_uint, p], i32),
             "w4a8_gemm_workspace_bytes": ([i32, i32, i32], sz),
             "w4a8_workspace_init": ([p, sz, p], i32),
             "w4a8_gemm": ([p, p, p, i32, i32, i32, p, p, sz, p], i32),
@@ -158,15 +162,20 @@ def w4a8_unpack_weights(packed, stream=None):
     return dict(codes=codes, s_u8=s, a=a, s_w=sw)
 
 
-def w4a8_quantize_act(X, out=None, scale_out=None, stream=None):
-    """Per-token INT8 quantization of fp32 X [M, K]: returns (Xq int8, s_x fp32)."""
+def w4a8_quantize_act(X, out=None, scale_out=None, stream=None, flags=0):
+    """Per-token INT8 quantization of fp32 X [M, K]: returns (Xq int8, s_x fp32).
+    ``flags`` are the launch options of w4a8_quantize_act_ex (0 = plain call)."""
     _need(X, _torch.float32, 2, "X")
     M, K = X.shape
     Xq = out if out is not None else _torch.empty(M, K, dtype=_torch.int8, device=X.device)
     sx = scale_out if scale_out is not None else _torch.empty(M, dtype=_torch.float32,
                                                               device=X.device)
-    _check(lib().w4a8_quantize_act(_ptr(X), M, K, _ptr(Xq), _ptr(sx), _stream(stream)),
-           "w4a8_quantize_act")
+    if flags:
+        rc = lib().w4a8_quantize_act_ex(_ptr(X), M, K, _ptr(Xq), _ptr(sx), int(flags),
+                                        _stream(stream))
+    else:
+        rc = lib().w4a8_quantize_act(_ptr(X), M, K, _ptr(Xq), _ptr(sx), _stream(stream))
+    _check(rc, "w4a8_quantize_act")
     return Xq, sx
 
 
@@ -199,8 +208,9 @@ def workspace_for(M, N, K, device=None, stream=None):
     return ws
 
 
-def w4a8_gemm(Xq, s_x, packed, out=None, workspace=None, stream=None):
-    """Y [M, N] bf16 = (s_x[m] s_w[n]) * sum_k Xq[m,k] Wdq[n,k]."""
+def w4a8_gemm(Xq, s_x, packed, out=None, workspace=None, stream=None, flags=0):
+    """Y [M, N] bf16 = (s_x[m] s_w[n]) * sum_k Xq[m,k] Wdq[n,k].
+    ``flags`` are the launch options of w4a8_gemm_ex (0 = plain call)."""
     _need(Xq, _torch.int8, 2, "Xq")
     _need(s_x, _torch.float32, 1, "s_x")
     M, K = Xq.shape
@@ -209,8 +219,14 @@ def w4a8_gemm(Xq, s_x, packed, out=None, workspace=None, stream=None):
     N = packed.N
     Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
     ws = workspace if workspace is not None else workspace_for(M, N, K, Xq.device, stream)
-    _check(lib().w4a8_gemm(_ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y), _ptr(ws),
-                           0 if ws is None else ws.numel(), _stream(stream)), "w4a8_gemm")
+    wsb = 0 if ws is None else ws.numel()
+    if flags:
+        rc = lib().w4a8_gemm_ex(_ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
+                                _ptr(ws), wsb, int(flags), _stream(stream))
+    else:
+        rc = lib().w4a8_gemm(_ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
+                             _ptr(ws), wsb, _stream(stream))
+    _check(rc, "w4a8_gemm")
     return Y
 
 

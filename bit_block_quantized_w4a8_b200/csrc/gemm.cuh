@@ -48,7 +48,7 @@ struct GemmParams {
   const float* s_x;       // per-token scales [M] (bf16 output only)
   uint16_t* Y;            // [M][N] bf16 bits, or nullptr
   int32_t* acc;           // [M][N] int32, or nullptr
-  int32_t* ws;            // split-K partials [m_tiles][n_pad][T]
+  int32_t* ws;            // split-K partials [m_tiles][T][n_pad]
   uint32_t* counters;     // split-K arrivals [m_tiles][n_tiles]
   int M, N, K, n_pad;
   int kt_total;           // K / 128
@@ -149,14 +149,11 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
     tmem_relinquish();
   }
-  if (p.Y) {
-    for (int i = threadIdx.x; i < T; i += C::kThreads)
-      sx_s[i] = (m0 + i < p.M) ? p.s_x[m0 + i] : 0.0f;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -165,7 +162,21 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
       const uint64_t pol = l2_policy_evict_first();
       const uint8_t* wsrc = p.tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
       int issued = 0;
-      for (int it = 0; it < nk; ++it) {
+      // The packed weights do not depend on the preceding kernel: the first
+      // ring's worth of weight tiles is requested before waiting for it.
+      const int pre = nk < STAGES ? nk : STAGES;
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(bar_full + 8 * it, C::kTxBytes);
+        bulk_g2s(sbase + C::kOffW + it * kTileBytes, wsrc + (size_t)it * kTileBytes,
+                 kTileBytes, bar_full + 8 * it, pol);
+      }
+      pdl_wait();  // activations are produced by the preceding kernel
+      for (int it = 0; it < pre; ++it) {
+        tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
+                    bar_full + 8 * it);
+        issued = it + 1;
+      }
+      for (int it = pre; it < nk; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
@@ -208,6 +219,13 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
     const int quarter = warp & 3;          // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;     // weight row in the tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int n = n_tile * kTileN + r;
+    // loads needed only by the epilogue, issued before the main loop so
+    // their latency is hidden
+    const float swn = n < p.N ? __ldg(p.s_w + n) : 0.0f;
+    bool hdr_ok = true;
+    if (warp == 2 && lane == 0)
+      hdr_ok = p.hdr->magic == kMagic && p.hdr->N == p.N && p.hdr->K == p.K;
     for (int it = dg; it < nk; it += DQG) {
       const int s = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
@@ -236,9 +254,12 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
 
     // -------------------------------------------------------- epilogue
     const int nthr = 128 * DQG;
-    bool hdr_ok = true;
-    if (warp == 2 && lane == 0)
-      hdr_ok = p.hdr->magic == kMagic && p.hdr->N == p.N && p.hdr->K == p.K;
+    pdl_wait();  // s_x, the workspace and Y belong to the preceding kernels' order
+    if (p.Y) {
+      const int et = threadIdx.x - 64;  // epilogue thread index
+      for (int i = et; i < T; i += nthr)
+        sx_s[i] = (m0 + i < p.M) ? p.s_x[m0 + i] : 0.0f;
+    }
     warp_wait(bar_acc, 0, abort_flag, lim);
     tc_fence_after();
     // one thread turns the abort flag into a value every epilogue thread
@@ -249,10 +270,8 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
       *ep_flag = (*abort_flag || !hdr_ok) ? 0 : 1;
     }
     named_bar_sync(1, nthr);
-    const int n = n_tile * kTileN + r;
     if (*ep_flag) {
       if (p.splits == 1) {
-        const float swn = n < p.N ? p.s_w[n] : 0.0f;
         for (int j = dg; j < T / 16; j += DQG) {
           uint32_t v[16];
           tmem_ld_x16(lane_base + 16 * j, v);
@@ -274,14 +293,17 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
           }
         }
       } else {
-        int32_t* wrow = p.ws + ((size_t)m_tile * p.n_pad + n) * T;
+        // partials are token-major ([token][channel]) so that for each token
+        // a warp's 32 reductions hit one contiguous 128-byte line
+        int32_t* wtile = p.ws + (size_t)m_tile * T * p.n_pad + n;
         for (int j = dg; j < T / 16; j += DQG) {
           uint32_t v[16];
           tmem_ld_x16(lane_base + 16 * j, v);
           tmem_wait_ld();
 #pragma unroll
           for (int t = 0; t < 16; ++t)
-            if (m0 + 16 * j + t < p.M) red_add_s32(wrow + 16 * j + t, (int32_t)v[t]);
+            if (m0 + 16 * j + t < p.M)
+              red_add_s32(wtile + (size_t)(16 * j + t) * p.n_pad, (int32_t)v[t]);
         }
         __threadfence();
         named_bar_sync(1, nthr);
@@ -293,20 +315,22 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
         named_bar_sync(1, nthr);
         if (*last_flag) {
           __threadfence();
-          const float swn = n < p.N ? p.s_w[n] : 0.0f;
           for (int j = dg; j < T / 16; j += DQG) {
+            int32_t a[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              a[t] = (m0 + 16 * j + t < p.M) ? __ldcg(wtile + (size_t)(16 * j + t) * p.n_pad) : 0;
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
               const int m = m0 + 16 * j + t;
               if (m < p.M) {
-                const int32_t a = __ldcg(wrow + 16 * j + t);
-                __stcg(wrow + 16 * j + t, 0);
+                __stcg(wtile + (size_t)(16 * j + t) * p.n_pad, 0);
                 if (n < p.N) {
                   if (p.Y) {
-                    const float y = (float)a * (sx_s[16 * j + t] * swn);
+                    const float y = (float)a[t] * (sx_s[16 * j + t] * swn);
                     p.Y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
                   } else {
-                    p.acc[(size_t)m * p.N + n] = a;
+                    p.acc[(size_t)m * p.N + n] = a[t];
                   }
                 }
               }

@@ -14,6 +14,7 @@
 #pragma once
 #include <cstdint>
 #include "layout.cuh"
+#include "ptx.cuh"
 
 namespace w4a8 {
 
@@ -177,10 +178,23 @@ __global__ void __launch_bounds__(128) weight_unpack_kernel(
   }
 }
 
-// Per-token activation quantization: one CTA per token row.  Pass 1 finds
-// the row's absmax, pass 2 (re-reading the row, now in L1/L2) writes the
-// INT8 codes four at a time.
+// Per-token activation quantization: one CTA per token row.  The first
+// kActRegs * kActThreads float4 of the row stay in registers between the
+// absmax pass and the quantization pass (the whole row for K <= 8192); the
+// rest of a longer row is read again (from L1/L2).
 constexpr int kActThreads = 256;
+constexpr int kActRegs = 8;
+
+__device__ __forceinline__ uint32_t quant4(float4 v, float s) {
+  return (uint32_t)(quant_sym(v.x, s, 127) & 0xFF) |
+         ((uint32_t)(quant_sym(v.y, s, 127) & 0xFF) << 8) |
+         ((uint32_t)(quant_sym(v.z, s, 127) & 0xFF) << 16) |
+         ((uint32_t)(quant_sym(v.w, s, 127) & 0xFF) << 24);
+}
+
+__device__ __forceinline__ float absmax4(float4 v) {
+  return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+}
 
 __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
     const float* __restrict__ X, int M, int K, int8_t* __restrict__ Xq,
@@ -189,32 +203,37 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
   const int m = blockIdx.x;
   const float4* row = reinterpret_cast<const float4*>(X + (size_t)m * K);
   const int n4 = K / 4;
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  pdl_wait();  // X may be produced by the preceding kernel
+  float4 v[kActRegs];
   float amax = 0.0f;
-  for (int i = threadIdx.x; i < n4; i += kActThreads) {
-    float4 v = __ldg(row + i);
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)),
-                             fmaxf(fabsf(v.z), fabsf(v.w))));
+#pragma unroll
+  for (int i = 0; i < kActRegs; ++i) {
+    const int idx = threadIdx.x + i * kActThreads;
+    v[i] = idx < n4 ? __ldg(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    amax = fmaxf(amax, absmax4(v[i]));
   }
+  for (int idx = threadIdx.x + kActRegs * kActThreads; idx < n4; idx += kActThreads)
+    amax = fmaxf(amax, absmax4(__ldg(row + idx)));
   amax = warp_max(amax);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
   __syncthreads();
   if (threadIdx.x < 32) {
-    float v = threadIdx.x < kActThreads / 32 ? red[threadIdx.x] : 0.0f;
-    v = warp_max(v);
-    if (threadIdx.x == 0) red[0] = v;
+    float r = threadIdx.x < kActThreads / 32 ? red[threadIdx.x] : 0.0f;
+    r = warp_max(r);
+    if (threadIdx.x == 0) red[0] = r;
   }
   __syncthreads();
   const float s = __fdiv_rn(red[0], 127.0f);
   if (threadIdx.x == 0) s_x[m] = s;
   uint32_t* out = reinterpret_cast<uint32_t*>(Xq + (size_t)m * K);
-  for (int i = threadIdx.x; i < n4; i += kActThreads) {
-    float4 v = __ldg(row + i);
-    uint32_t q = (uint32_t)(quant_sym(v.x, s, 127) & 0xFF) |
-                 ((uint32_t)(quant_sym(v.y, s, 127) & 0xFF) << 8) |
-                 ((uint32_t)(quant_sym(v.z, s, 127) & 0xFF) << 16) |
-                 ((uint32_t)(quant_sym(v.w, s, 127) & 0xFF) << 24);
-    out[i] = q;
+#pragma unroll
+  for (int i = 0; i < kActRegs; ++i) {
+    const int idx = threadIdx.x + i * kActThreads;
+    if (idx < n4) out[idx] = quant4(v[i], s);
   }
+  for (int idx = threadIdx.x + kActRegs * kActThreads; idx < n4; idx += kActThreads)
+    out[idx] = quant4(__ldg(row + idx), s);
 }
 
 }  // namespace w4a8

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "gemm.cuh"
 #include "layout.cuh"
@@ -114,9 +115,26 @@ size_t workspace_bytes_for(const Schedule& s, int N) {
 }
 
 // ------------------------------------------------------------- launches
+// Launch with or without programmatic dependent launch (PDL).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
 template <int T, int STAGES, int DQG, int MINB>
 cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
-                        cudaStream_t st) {
+                        cudaStream_t st, bool pdl) {
   using C = GemmCfg<T, STAGES, DQG>;
   auto k = w4a8_gemm_kernel<T, STAGES, DQG, MINB>;
   static std::atomic<bool> attr_set[kMaxDevices];
@@ -127,13 +145,14 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_relaxed);
   }
-  k<<<ctas, C::kThreads, C::kSmemBytes, st>>>(map, p);
-  return cudaGetLastError();
+  return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, map, p);
 }
 
 int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
                 int K, uint16_t* Y, int32_t* acc, void* workspace, size_t ws_bytes,
-                void* stream) {
+                unsigned flags, void* stream) {
+  if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
+  const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
   if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
   if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return W4A8_OK;
@@ -177,11 +196,11 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
   switch (s.T) {
-    case 16: e = launch_gemm<16, 6, 2, 2>(map, p, s.ctas, st); break;
-    case 32: e = launch_gemm<32, 6, 2, 2>(map, p, s.ctas, st); break;
-    case 64: e = launch_gemm<64, 6, 2, 2>(map, p, s.ctas, st); break;
-    case 128: e = launch_gemm<128, 4, 2, 2>(map, p, s.ctas, st); break;
-    default: e = launch_gemm<256, 5, 2, 1>(map, p, s.ctas, st); break;
+    case 16: e = launch_gemm<16, 6, 2, 2>(map, p, s.ctas, st, pdl); break;
+    case 32: e = launch_gemm<32, 6, 2, 2>(map, p, s.ctas, st, pdl); break;
+    case 64: e = launch_gemm<64, 6, 2, 2>(map, p, s.ctas, st, pdl); break;
+    case 128: e = launch_gemm<128, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
+    default: e = launch_gemm<256, 5, 2, 1>(map, p, s.ctas, st, pdl); break;
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
@@ -265,13 +284,20 @@ int w4a8_unpack_weights(const void* packed, int N, int K, uint8_t* codes, uint8_
 }
 
 int w4a8_quantize_act(const float* X, int M, int K, int8_t* Xq, float* s_x, void* stream) {
+  return w4a8_quantize_act_ex(X, M, K, Xq, s_x, 0u, stream);
+}
+
+int w4a8_quantize_act_ex(const float* X, int M, int K, int8_t* Xq, float* s_x, unsigned flags,
+                         void* stream) {
+  if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
   if (M < 0 || K < 1) return W4A8_ERR_INVALID_ARG;
   if (K % 16 != 0) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return W4A8_OK;
   if (!X || !Xq || !s_x) return W4A8_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(s_x, 4)) return W4A8_ERR_MISALIGNED;
-  act_quant_kernel<<<M, kActThreads, 0, as_stream(stream)>>>(X, M, K, Xq, s_x);
-  return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+  cudaError_t e = launch_k(act_quant_kernel, dim3(M), dim3(kActThreads), 0, as_stream(stream),
+                           (flags & W4A8_FLAG_PDL) != 0, X, M, K, Xq, s_x);
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
 size_t w4a8_gemm_workspace_bytes(int M, int N, int K) {
@@ -290,12 +316,17 @@ int w4a8_workspace_init(void* workspace, size_t bytes, void* stream) {
 
 int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M, int N, int K,
               uint16_t* Y, void* workspace, size_t ws_bytes, void* stream) {
-  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, workspace, ws_bytes, stream);
+  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, workspace, ws_bytes, 0u, stream);
+}
+
+int w4a8_gemm_ex(const int8_t* Xq, const float* s_x, const void* packed, int M, int N, int K,
+                 uint16_t* Y, void* workspace, size_t ws_bytes, unsigned flags, void* stream) {
+  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, workspace, ws_bytes, flags, stream);
 }
 
 int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K, int32_t* acc,
                   void* workspace, size_t ws_bytes, void* stream) {
-  return gemm_common(Xq, nullptr, packed, M, N, K, nullptr, acc, workspace, ws_bytes,
+  return gemm_common(Xq, nullptr, packed, M, N, K, nullptr, acc, workspace, ws_bytes, 0u,
                      stream);
 }
 

@@ -144,6 +144,28 @@ int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M,
               int N, int K, uint16_t* Y, void* workspace, size_t ws_bytes,
               void* stream);
 
+/*
+ * Launch options for the *_ex entry points (bit mask).
+ * W4A8_FLAG_PDL: launch with programmatic dependent launch.  The kernel may
+ *   start while the kernel before it in the stream is still running; it
+ *   waits for that kernel's results before reading its activation inputs or
+ *   writing anything, but it reads the packed weights (and their scales)
+ *   early.  Use it only when the preceding kernel in the stream does not
+ *   write the packed weight buffer.  This hides launch and weight-fetch
+ *   latency in chains of small calls (decode).
+ */
+#define W4A8_FLAG_PDL 1u
+
+/* w4a8_gemm with launch options (flags as above; 0 = w4a8_gemm). */
+int w4a8_gemm_ex(const int8_t* Xq, const float* s_x, const void* packed, int M,
+                 int N, int K, uint16_t* Y, void* workspace, size_t ws_bytes,
+                 unsigned flags, void* stream);
+
+/* w4a8_quantize_act with launch options (flags as above).  With
+ * W4A8_FLAG_PDL it waits for the preceding kernel before reading X. */
+int w4a8_quantize_act_ex(const float* X, int M, int K, int8_t* Xq, float* s_x,
+                         unsigned flags, void* stream);
+
 /* Same product, writing the exact INT32 accumulators acc [M][N] instead of
  * the bf16 output (for bit-exact verification). */
 int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K,

@@ -229,3 +229,30 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert w4.w4a8_get_status() == 0
     acc, y, acc_ref, y_ref, _ = _run_case(3, 128, 256, seed=5)
     assert np.array_equal(acc, acc_ref)
+
+
+def test_pdl_chain_matches_plain_calls():
+    """Chains of quantize -> GEMM launched with programmatic dependent launch
+    (each kernel may start while the previous one finishes) give the same
+    bits as plain launches, including split-K shapes sharing one workspace."""
+    K = 2048
+    W = wl.random_matrix(256, K, 41, std=0.02).cuda()
+    pk = w4.w4a8_quantize_weights(W)
+    Ms = [1, 3, 16, 40, 130, 300]
+    Xs = [wl.random_matrix(M, K, 50 + M).cuda() for M in Ms]
+    ws = torch.zeros(max(w4.w4a8_gemm_workspace_bytes(M, 256, K) for M in Ms) + 256,
+                     dtype=torch.uint8, device="cuda")
+    ref = []
+    for X in Xs:
+        xq, s = w4.w4a8_quantize_act(X)
+        ref.append(w4.w4a8_gemm(xq, s, pk, workspace=ws).clone())
+    for rep in range(3):
+        outs = []
+        for X in Xs:
+            xq, s = w4.w4a8_quantize_act(X, flags=w4.W4A8_FLAG_PDL)
+            outs.append(w4.w4a8_gemm(xq, s, pk, workspace=ws, flags=w4.W4A8_FLAG_PDL))
+        torch.cuda.synchronize()
+        for a, b in zip(outs, ref):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert w4.w4a8_get_status() == 0
+    assert ws_is_zero(ws)
