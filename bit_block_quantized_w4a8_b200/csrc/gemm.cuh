@@ -229,9 +229,14 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
     for (int it = dg; it < nk; it += DQG) {
       const int s = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
-      if (!warp_wait(bar_full + 8 * s, ph, abort_flag, lim)) break;
-      // the MMAs of the previous round of this slot are done (TMEM A free)
+      // First the previous round of this slot must be fully consumed (its
+      // MMAs done, so its TMEM A columns are free).  Only then is the parity
+      // wait on the full barrier unambiguous: a group skips the other
+      // group's iterations, so it can reach round k of a slot while round
+      // k-1's copies are still in flight; the barrier's last completed phase
+      // is then k-2, whose parity equals k's, and a parity wait would pass.
       if (!warp_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
+      if (!warp_wait(bar_full + 8 * s, ph, abort_flag, lim)) break;
       tc_fence_after();
       const uint32_t wbase = sbase + C::kOffW + s * kTileBytes;
       const uint32_t prm = lds32(wbase + kCodeBytes + 4 * r);

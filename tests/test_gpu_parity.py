@@ -256,3 +256,37 @@ def test_pdl_chain_matches_plain_calls():
             assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert w4.w4a8_get_status() == 0
     assert ws_is_zero(ws)
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 4096, 4096), (1024, 8192, 2048), (48, 2048, 8192)])
+def test_repeated_runs_deep_k(M, N, K):
+    """Many ring rounds per CTA, repeated: every run bit-identical, and exact
+    against the oracle on sampled outputs plus row/column-sum invariants over
+    all outputs (guards the pipeline's barrier protocol)."""
+    X = wl.random_matrix(M, K, 71 + M, std=1.0, kind="heavy")
+    W = wl.random_matrix(N, K, 72 + N, std=0.02)
+    Xq_ref, sx_ref = oracle.quantize_act(X.numpy())
+    wq = _oracle_weights(W)
+    W8 = oracle.dequant_weights(wq["codes"], wq["s_u8"], wq["a"])
+    pk = w4.w4a8_quantize_weights(W.cuda())
+    Xq, sx = w4.w4a8_quantize_act(X.cuda())
+    ws = w4.workspace_for(M, N, K)
+    first = None
+    rng = np.random.default_rng(M + N + K)
+    ms = rng.integers(0, M, 256)
+    ns = rng.integers(0, N, 256)
+    acc_s_ref, _ = oracle.w4a8_gemm_sampled(Xq_ref, sx_ref, wq, ms, ns)
+    row_ref = Xq_ref.astype(np.int64) @ W8.sum(axis=0, dtype=np.int64)
+    col_ref = W8.astype(np.int64) @ Xq_ref.sum(axis=0, dtype=np.int64)
+    for rep in range(6):
+        acc = w4.w4a8_gemm_i32(Xq, pk, workspace=ws)
+        torch.cuda.synchronize()
+        assert w4.w4a8_get_status() == 0
+        if first is None:
+            first = acc.clone()
+            assert np.array_equal(acc.cpu().numpy()[ms, ns], acc_s_ref)
+            assert np.array_equal(acc.sum(dim=1, dtype=torch.int64).cpu().numpy(), row_ref)
+            assert np.array_equal(acc.sum(dim=0, dtype=torch.int64).cpu().numpy(), col_ref)
+        else:
+            assert torch.equal(acc, first), "run %d differs from run 0" % rep
+    assert ws_is_zero(ws)
