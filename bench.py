@@ -337,8 +337,6 @@ def run_cuda(args):
     Xq = {M: torch.empty(M, K, dtype=torch.int8, device=dev) for M in Ms}
     sx = {M: torch.empty(M, dtype=torch.float32, device=dev) for M in Ms}
     Ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in Ms}
-    ws_need = max(w4.w4a8_gemm_workspace_bytes(M, N, K) for M in Ms)
-    ws = torch.zeros(max(ws_need, 256), dtype=torch.uint8, device=dev)
 
     stream = torch.cuda.Stream(device=dev)
 
@@ -348,7 +346,7 @@ def run_cuda(args):
                 w4.w4a8_quantize_act(Xs[M], out=Xq[M], scale_out=sx[M], stream=stream,
                                      flags=PDL)
                 w4.w4a8_gemm(Xq[M], sx[M], copies[(r * len(Ms) + j) % N_COPIES], out=Ys[M],
-                             workspace=ws, stream=stream, flags=PDL)
+                             stream=stream, flags=PDL)
         return fn
 
     with torch.cuda.stream(stream):
@@ -394,8 +392,7 @@ def run_cuda(args):
     for M in Ms:
         def gemms(M=M, fl=PDL):
             for i in range(N_COPIES):
-                w4.w4a8_gemm(Xq[M], sx[M], copies[i], out=Ys[M], workspace=ws, stream=stream,
-                             flags=fl)
+                w4.w4a8_gemm(Xq[M], sx[M], copies[i], out=Ys[M], stream=stream, flags=fl)
 
         def quants(M=M):
             for i in range(N_COPIES):
@@ -448,7 +445,7 @@ def run_cuda(args):
             xq, s_ = w4.w4a8_quantize_act(dX[M], out=Xq[M], scale_out=sx[M], stream=stream,
                                           flags=PDL)
             y = w4.w4a8_gemm(xq, s_, copies[(r * len(Ms) + j) % N_COPIES], out=Ys[M],
-                             workspace=ws, stream=stream, flags=PDL)
+                             stream=stream, flags=PDL)
             hY[M].copy_(y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -518,6 +515,82 @@ def run_profile_case(args):
     return 0 if status == 0 else 1
 
 
+def run_all_configs(args):
+    """Kernel timings on every synthetic workload (all layers and M values):
+    per case the GEMM and the activation quantizer are each timed as graphs
+    of back-to-back launches (programmatic dependent launch), with enough
+    rotating weight copies that the working set exceeds twice the L2.
+    Writes one JSON document to ``args.all_configs``."""
+    import bit_block_quantized_w4a8_b200 as w4
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    out = {"peaks": peaks, "cases": []}
+    for name in wl.WORKLOADS:
+        layers_done = {}
+        for M, layer in wl.cases(name):
+            N, K = layer.N, layer.K
+            if layer.name not in layers_done:
+                layers_done.clear()
+                torch.cuda.empty_cache()
+                W = wl.layer_weights(name, layer).to(dev)
+                pk = w4.w4a8_quantize_weights(W)
+                del W
+                ncopy = max(1, min(32, -(-2 * l2 // pk.data.numel())))
+                copies = [pk] + [w4.PackedWeights(pk.data.clone(), N, K, GROUP)
+                                 for _ in range(ncopy - 1)]
+                layers_done[layer.name] = copies
+            copies = layers_done[layer.name]
+            X = wl.layer_activations(name, layer, M).to(dev)
+            Xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+            sx = torch.empty(M, dtype=torch.float32, device=dev)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            reps_in = max(len(copies), 4)
+            with torch.cuda.stream(stream):
+                w4.w4a8_quantize_act(X, out=Xq, scale_out=sx, stream=stream)
+                w4.w4a8_gemm(Xq, sx, copies[0], out=Y, stream=stream)
+            stream.synchronize()
+
+            def gemms():
+                for i in range(reps_in):
+                    w4.w4a8_gemm(Xq, sx, copies[i % len(copies)], out=Y, stream=stream,
+                                 flags=PDL)
+
+            def quants():
+                for i in range(reps_in):
+                    w4.w4a8_quantize_act(X, out=Xq, scale_out=sx, stream=stream, flags=PDL)
+            gg, gq = _graph(gemms, stream), _graph(quants, stream)
+            with torch.cuda.stream(stream):
+                gg.replay()
+                gq.replay()
+            reps = max(3, min(50, int(2e-3 / max(1e-6, _time_graph(gg, 1, stream)))))
+            tg = _time_graph(gg, reps, stream) / reps_in
+            tq = _time_graph(gq, reps, stream) / reps_in
+            status = w4.w4a8_get_status(stream)
+            b, o = gemm_bytes(M, N, K), gemm_ops(M, N, K)
+            hbm_t, tc_t = b / (peaks["hbm"] * 1e9), o / (peaks["bf16"] * INT8_PER_BF16 * 1e12)
+            bound = "hbm" if hbm_t >= tc_t else "tensor"
+            T, splits, ctas = w4.w4a8_gemm_schedule(M, N, K)
+            case = {"workload": name, "layer": layer.name, "M": M, "N": N, "K": K,
+                    "gemm_us": tg * 1e6, "tops": o / tg / 1e12,
+                    "weight_gbs": weight_bytes(N, K) / tg / 1e9, "total_gbs": b / tg / 1e9,
+                    "bound": bound, "frac": (hbm_t if bound == "hbm" else tc_t) / tg,
+                    "act_quant_us": tq * 1e6, "act_quant_gbs": act_bytes(M, K) / tq / 1e9,
+                    "weight_copies": len(copies), "status": status,
+                    "schedule": {"tile_tokens": T, "splits": splits, "ctas": ctas}}
+            out["cases"].append(case)
+            print("%-18s %-9s M=%-6d %9.2f us %8.1f TOPS %7.0f wGB/s %-6s %.3f  (%s)" % (
+                name, layer.name, M, case["gemm_us"], case["tops"], case["weight_gbs"], bound,
+                case["frac"], case["schedule"]), flush=True)
+            del gg, gq
+        layers_done.clear()
+    with open(args.all_configs, "w") as f:
+        json.dump(out, f, indent=1)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,7 +602,11 @@ def main(argv=None):
                     help="seconds of CPU work for the oracle baseline sample")
     ap.add_argument("--profile", default=None,
                     help="comma-separated Ms: run one GEMM each on N=K=4096 for a profiler")
+    ap.add_argument("--all-configs", default=None, metavar="PATH",
+                    help="time every workload case and write a JSON report to PATH")
     args = ap.parse_args(argv)
+    if args.all_configs:
+        return run_all_configs(args)
     if args.profile:
         return run_profile_case(args)
     if args.warmup < 3:

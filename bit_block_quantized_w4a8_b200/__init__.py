@@ -22,16 +22,14 @@ from .build import LIB as _LIB_PATH
 __all__ = [
     "W4A8Error", "lib", "w4a8_version", "w4a8_status_string",
     "w4a8_packed_weight_bytes", "w4a8_quantize_weights", "w4a8_unpack_weights",
-    "w4a8_quantize_act", "w4a8_gemm_workspace_bytes", "w4a8_workspace_init",
-    "w4a8_gemm", "w4a8_gemm_i32", "w4a8_gemm_schedule", "w4a8_get_status",
-    "w4a8_debug_timeout_probe", "PackedWeights", "workspace_for",
+    "w4a8_quantize_act", "w4a8_gemm", "w4a8_gemm_i32", "w4a8_gemm_schedule",
+    "w4a8_get_status", "w4a8_debug_timeout_probe", "PackedWeights",
 ]
 
 OK = 0
 ERR_INVALID_ARG = -1
 ERR_UNSUPPORTED_SHAPE = -2
 ERR_MISALIGNED = -3
-ERR_WORKSPACE = -4
 ERR_CUDA = -5
 ERR_TIMEOUT = -6
 ERR_BAD_PACKED = -7
@@ -71,11 +69,9 @@ def lib():
             "w4a8_unpack_weights": ([p, i32, i32, p, p, p, p, p], i32),
             "w4a8_quantize_act": ([p, i32, i32, p, p, p], i32),
             "w4a8_quantize_act_ex": ([p, i32, i32, p, p, _ct.c_uint, p], i32),
-            "w4a8_gemm_ex": ([p, p, p, i32, i32, i32, p, p, sz, _ct.c_uint, p], i32),
-            "w4a8_gemm_workspace_bytes": ([i32, i32, i32], sz),
-            "w4a8_workspace_init": ([p, sz, p], i32),
-            "w4a8_gemm": ([p, p, p, i32, i32, i32, p, p, sz, p], i32),
-            "w4a8_gemm_i32": ([p, p, i32, i32, i32, p, p, sz, p], i32),
+            "w4a8_gemm_ex": ([p, p, p, i32, i32, i32, p, _ct.c_uint, p], i32),
+            "w4a8_gemm": ([p, p, p, i32, i32, i32, p, p], i32),
+            "w4a8_gemm_i32": ([p, p, i32, i32, i32, p, p], i32),
             "w4a8_gemm_schedule": ([i32, i32, i32, p, p, p], i32),
             "w4a8_get_status": ([p], i32),
             "w4a8_debug_timeout_probe": ([ll, p], i32),
@@ -179,36 +175,7 @@ def w4a8_quantize_act(X, out=None, scale_out=None, stream=None, flags=0):
     return Xq, sx
 
 
-def w4a8_gemm_workspace_bytes(M, N, K):
-    return int(lib().w4a8_gemm_workspace_bytes(int(M), int(N), int(K)))
-
-
-def w4a8_workspace_init(ws, stream=None):
-    _check(lib().w4a8_workspace_init(_ptr(ws), ws.numel(), _stream(stream)),
-           "w4a8_workspace_init")
-
-
-_ws_cache = {}
-
-
-def workspace_for(M, N, K, device=None, stream=None):
-    """A zero-filled workspace big enough for (M, N, K), cached per device and
-    stream (calls on one stream run in order, so they may share it)."""
-    need = w4a8_gemm_workspace_bytes(M, N, K)
-    if need == 0:
-        return None
-    dev = _torch.device(device) if device is not None else _torch.device(
-        "cuda", _torch.cuda.current_device())
-    s = stream if stream is not None else _torch.cuda.current_stream(dev)
-    key = (dev.index, s.cuda_stream)
-    ws = _ws_cache.get(key)
-    if ws is None or ws.numel() < need:
-        ws = _torch.zeros(max(need, 1 << 20), dtype=_torch.uint8, device=dev)
-        _ws_cache[key] = ws
-    return ws
-
-
-def w4a8_gemm(Xq, s_x, packed, out=None, workspace=None, stream=None, flags=0):
+def w4a8_gemm(Xq, s_x, packed, out=None, stream=None, flags=0):
     """Y [M, N] bf16 = (s_x[m] s_w[n]) * sum_k Xq[m,k] Wdq[n,k].
     ``flags`` are the launch options of w4a8_gemm_ex (0 = plain call)."""
     _need(Xq, _torch.int8, 2, "Xq")
@@ -218,19 +185,17 @@ def w4a8_gemm(Xq, s_x, packed, out=None, workspace=None, stream=None, flags=0):
         raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
     N = packed.N
     Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
-    ws = workspace if workspace is not None else workspace_for(M, N, K, Xq.device, stream)
-    wsb = 0 if ws is None else ws.numel()
     if flags:
         rc = lib().w4a8_gemm_ex(_ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
-                                _ptr(ws), wsb, int(flags), _stream(stream))
+                                int(flags), _stream(stream))
     else:
         rc = lib().w4a8_gemm(_ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
-                             _ptr(ws), wsb, _stream(stream))
+                             _stream(stream))
     _check(rc, "w4a8_gemm")
     return Y
 
 
-def w4a8_gemm_i32(Xq, packed, out=None, workspace=None, stream=None):
+def w4a8_gemm_i32(Xq, packed, out=None, stream=None):
     """Exact INT32 accumulators acc [M, N] = sum_k Xq[m,k] Wdq[n,k]."""
     _need(Xq, _torch.int8, 2, "Xq")
     M, K = Xq.shape
@@ -238,10 +203,8 @@ def w4a8_gemm_i32(Xq, packed, out=None, workspace=None, stream=None):
         raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
     N = packed.N
     acc = out if out is not None else _torch.empty(M, N, dtype=_torch.int32, device=Xq.device)
-    ws = workspace if workspace is not None else workspace_for(M, N, K, Xq.device, stream)
-    _check(lib().w4a8_gemm_i32(_ptr(Xq), _ptr(packed.data), M, N, K, _ptr(acc), _ptr(ws),
-                               0 if ws is None else ws.numel(), _stream(stream)),
-           "w4a8_gemm_i32")
+    _check(lib().w4a8_gemm_i32(_ptr(Xq), _ptr(packed.data), M, N, K, _ptr(acc),
+                               _stream(stream)), "w4a8_gemm_i32")
     return acc
 
 

@@ -21,15 +21,21 @@
 //     tcgen05.st per 32 weights and thread.
 //   * Warp roles per CTA: warp 0 issues the copies (1-D bulk copy of a
 //     packed weight tile + 2-D TMA of the activation tile), warp 1 issues
-//     the MMAs (one thread), DQG groups of 4 warps dequantize (thread =
-//     weight row = TMEM lane) and then run the epilogue.
-//   * Ring of STAGES slots, each holding one weight tile and one
-//     activation tile in shared memory and one 32-column A slot in TMEM.
-//     Barriers per slot: full (copies landed), dq (A slot written), empty
-//     (MMAs that read the slot completed, via tcgen05.commit).
-//   * Split-K for few output tiles (decode): each split adds its INT32
-//     partials into a workspace with red.add; the last split to arrive (a
-//     per-tile counter) applies the epilogue and zeroes what it used.
+//     the MMAs, each through one elected lane of the converged warp; DQG
+//     groups of 4 warps dequantize (thread = weight row = TMEM lane) and
+//     then run the epilogue.
+//   * Two rings.  SS shared-memory stages each hold one packed weight tile
+//     and one activation tile (deep, to keep enough bytes in flight to
+//     cover DRAM latency); AS TMEM slots of 32 columns each hold one
+//     dequantized 128 x 128 weight tile (A operand).  Barriers: full[ss]
+//     (copies landed), empty[ss] (the MMAs that read the stage completed),
+//     dq[as] (A slot written), afree[as] (the MMAs that read the A slot
+//     completed); the completions come from tcgen05.commit.
+//   * Split-K for few output tiles (decode): the splits of one output tile
+//     form a thread-block cluster.  Each CTA leaves its INT32 partial tile
+//     in its own shared memory; after a cluster barrier every CTA sums one
+//     slice of the tile over all partials through distributed shared memory
+//     and applies the epilogue to it.  No global workspace, no atomics.
 //   * Every wait is bounded (globaltimer); a wait that runs out records a
 //     timeout in the device status word and all roles leave their loops,
 //     wait for their own copies / MMAs in flight, free TMEM and return.
@@ -48,35 +54,35 @@ struct GemmParams {
   const float* s_x;       // per-token scales [M] (bf16 output only)
   uint16_t* Y;            // [M][N] bf16 bits, or nullptr
   int32_t* acc;           // [M][N] int32, or nullptr
-  int32_t* ws;            // split-K partials [m_tiles][T][n_pad]
-  uint32_t* counters;     // split-K arrivals [m_tiles][n_tiles]
   int M, N, K, n_pad;
   int kt_total;           // K / 128
   int splits, kt_per_split;
   int n_tiles, m_tiles;
+  uint32_t x_tx_bytes;    // bytes of one activation box (rows * 128)
   unsigned long long wait_limit_ns;
   const PackedHeader* hdr;  // checked against (N, K) before any store
 };
 
-template <int T, int STAGES, int DQG>
+template <int T, int SS, int AS, int DQG>
 struct GemmCfg {
   static_assert(T % 16 == 0 && T >= 16 && T <= 256, "MMA N for M=128");
+  static_assert(AS <= SS, "the TMEM ring must not be deeper than the smem ring");
   static constexpr int kXBytes = T * kTileK;             // activation tile
-  static constexpr int kStageBytes = kXBytes + kTileBytes;
   static constexpr int kThreads = (2 + 4 * DQG) * 32;
   static constexpr int kA0 = T < 32 ? 32 : T;             // first A column
-  static constexpr int kColsUsed = kA0 + 32 * STAGES;
+  static constexpr int kColsUsed = kA0 + 32 * AS;
   static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
                                    : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
   static_assert(kColsUsed <= 512, "TMEM columns");
   // shared memory: x tiles | w tiles | barriers | misc | s_x cache
-  static constexpr int kOffW = STAGES * kXBytes;
-  static constexpr int kOffBar = kOffW + STAGES * kTileBytes;
-  static constexpr int kNumBars = 3 * STAGES + 1;
+  static constexpr int kOffW = SS * kXBytes;
+  static constexpr int kOffBar = kOffW + SS * kTileBytes;
+  static constexpr int kNumBars = 2 * SS + 2 * AS + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffSx = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffSx + 4 * T + 1024;  // + alignment slack
-  static constexpr uint32_t kTxBytes = kXBytes + kTileBytes;
+  // the split-K partial tile reuses the pipeline buffers
+  static_assert(T * kTileN * 4 <= kOffBar, "partial tile must fit the stage buffers");
 };
 
 // Dequantize four packed words (32 codes of one row, k order given by the
@@ -94,6 +100,18 @@ __device__ __forceinline__ void dequant_chunk(uint4 v, uint32_t s, uint32_t a4,
   }
 }
 
+// One output: bf16(acc * (s_x * s_w)) in fp32 with a single rounding, or
+// the exact INT32 accumulator.
+__device__ __forceinline__ void store_out(const GemmParams& p, int m, int n, int32_t a,
+                                          float sx, float sw) {
+  if (p.Y) {
+    const float y = (float)a * (sx * sw);
+    p.Y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+  } else {
+    p.acc[(size_t)m * p.N + n] = a;
+  }
+}
+
 // All 32 lanes wait; the warp proceeds only if every lane saw the phase
 // complete (keeps the .sync.aligned tcgen05 instructions warp-uniform).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
@@ -102,32 +120,33 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int T, int STAGES, int DQG, int MINB>
-__global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
+template <int T, int SS, int AS, int DQG, int MINB>
+__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const GemmParams p) {
-  using C = GemmCfg<T, STAGES, DQG>;
+  using C = GemmCfg<T, SS, AS, DQG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const uint32_t bar_full = sbase + C::kOffBar;        // + 8 s
-  const uint32_t bar_empty = bar_full + 8 * STAGES;    // + 8 s
-  const uint32_t bar_dq = bar_empty + 8 * STAGES;      // + 8 s
-  const uint32_t bar_acc = bar_dq + 8 * STAGES;
+  const uint32_t bar_full = sbase + C::kOffBar;     // + 8 ss
+  const uint32_t bar_empty = bar_full + 8 * SS;     // + 8 ss
+  const uint32_t bar_dq = bar_empty + 8 * SS;       // + 8 as
+  const uint32_t bar_afree = bar_dq + 8 * AS;       // + 8 as
+  const uint32_t bar_acc = bar_afree + 8 * AS;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
   volatile int* ep_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
   float* sx_s = reinterpret_cast<float*>(smem + C::kOffSx);
 
-  // tile coordinates: channel block fastest, then token block, then split
-  const int n_tile = blockIdx.x % p.n_tiles;
-  const int rest = blockIdx.x / p.n_tiles;
-  const int m_tile = rest % p.m_tiles;
-  const int split = rest / p.m_tiles;
+  // tile coordinates: the splits of a tile are consecutive blocks (one
+  // cluster), then channel blocks, then token blocks
+  const int split = blockIdx.x % p.splits;
+  const int tile = blockIdx.x / p.splits;
+  const int n_tile = tile % p.n_tiles;
+  const int m_tile = tile / p.n_tiles;
   const int kt0 = split * p.kt_per_split;
   const int kt1 = min(kt0 + p.kt_per_split, p.kt_total);
   const int nk = kt1 - kt0;
@@ -135,14 +154,16 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
   const uint64_t lim = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < SS; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
-      mbar_init(bar_dq + 8 * s, 4);
+    }
+    for (int a = 0; a < AS; ++a) {
+      mbar_init(bar_dq + 8 * a, 4);
+      mbar_init(bar_afree + 8 * a, 1);
     }
     mbar_init(bar_acc, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -157,62 +178,77 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmap_x);
-      const uint64_t pol = l2_policy_evict_first();
-      const uint8_t* wsrc = p.tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
-      int issued = 0;
-      // The packed weights do not depend on the preceding kernel: the first
-      // ring's worth of weight tiles is requested before waiting for it.
-      const int pre = nk < STAGES ? nk : STAGES;
+    // The whole warp runs the loop and waits; one elected lane issues the
+    // copies (a converged warp issues these single-thread instructions much
+    // faster than a lone diverged lane).
+    const bool leader = elect_one();
+    const uint32_t tx = kTileBytes + p.x_tx_bytes;
+    if (leader) prefetch_tensormap(&tmap_x);
+    const uint64_t pol = l2_policy_evict_first();
+    const uint8_t* wsrc = p.tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
+    int issued = 0;
+    // The packed weights do not depend on the preceding kernel: the first
+    // ring's worth of weight tiles is requested before waiting for it.
+    const int pre = nk < SS ? nk : SS;
+    if (leader) {
       for (int it = 0; it < pre; ++it) {
-        mbar_arrive_expect_tx(bar_full + 8 * it, C::kTxBytes);
+        mbar_arrive_expect_tx(bar_full + 8 * it, tx);
         bulk_g2s(sbase + C::kOffW + it * kTileBytes, wsrc + (size_t)it * kTileBytes,
                  kTileBytes, bar_full + 8 * it, pol);
       }
-      pdl_wait();  // activations are produced by the preceding kernel
-      for (int it = 0; it < pre; ++it) {
+    }
+    pdl_wait();  // activations are produced by the preceding kernel
+    if (leader) {
+      for (int it = 0; it < pre; ++it)
         tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
                     bar_full + 8 * it);
-        issued = it + 1;
-      }
-      for (int it = pre; it < nk; ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
-        mbar_arrive_expect_tx(bar_full + 8 * s, C::kTxBytes);
+    }
+    issued = pre;
+    __syncwarp();
+    for (int it = pre; it < nk; ++it) {
+      const int s = it % SS;
+      const uint32_t ph = (it / SS) & 1;
+      if (!warp_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
+      if (leader) {
+        mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         bulk_g2s(sbase + C::kOffW + s * kTileBytes, wsrc + (size_t)it * kTileBytes,
                  kTileBytes, bar_full + 8 * s, pol);
         tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
                     bar_full + 8 * s);
-        issued = it + 1;
       }
-      if (*abort_flag) {
-        // let the copies already issued land before the CTA goes away
-        for (int it = issued - STAGES < 0 ? 0 : issued - STAGES; it < issued; ++it)
-          mbar_wait(bar_full + 8 * (it % STAGES), (it / STAGES) & 1, nullptr, lim);
-      }
+      __syncwarp();
+      issued = it + 1;
     }
+    if (*abort_flag) {
+      // let the copies already issued land before the CTA goes away
+      for (int it = issued - SS < 0 ? 0 : issued - SS; it < issued; ++it)
+        mbar_wait(bar_full + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
+    }
+    __syncwarp();  // reconverge before any CTA- or cluster-wide barrier
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(128, T);
-      for (int it = 0; it < nk; ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        if (!mbar_wait(bar_dq + 8 * s, ph, abort_flag, lim)) break;
-        if (!mbar_wait(bar_full + 8 * s, ph, abort_flag, lim)) break;
-        tc_fence_after();
-        const uint32_t a_tmem = tmem + C::kA0 + 32 * s;
+    // Whole warp waits, one elected lane issues the MMAs and commits.
+    const bool leader = elect_one();
+    constexpr uint32_t idesc = idesc_i8(128, T);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % SS, a = it % AS;
+      if (!warp_wait(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
+      if (!warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t a_tmem = tmem + C::kA0 + 32 * a;
         const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
 #pragma unroll
         for (int kk = 0; kk < kTileK / 32; ++kk)
           mma_i8_ts(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc,
                     (it | kk) != 0);
         tc_commit(bar_empty + 8 * s);
+        tc_commit(bar_afree + 8 * a);
       }
-      tc_commit(bar_acc);  // also on abort: tracks every MMA issued
+      __syncwarp();
     }
+    if (leader) tc_commit(bar_acc);  // also on abort: tracks every MMA issued
+    __syncwarp();
   } else {
     // --------------------------------------------- dequantization warps
     const int dg = (warp - 2) / 4;         // dequant group
@@ -227,53 +263,57 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
     if (warp == 2 && lane == 0)
       hdr_ok = p.hdr->magic == kMagic && p.hdr->N == p.N && p.hdr->K == p.K;
     for (int it = dg; it < nk; it += DQG) {
-      const int s = it % STAGES;
-      const uint32_t ph = (it / STAGES) & 1;
-      // First the previous round of this slot must be fully consumed (its
-      // MMAs done, so its TMEM A columns are free).  Only then is the parity
-      // wait on the full barrier unambiguous: a group skips the other
-      // group's iterations, so it can reach round k of a slot while round
-      // k-1's copies are still in flight; the barrier's last completed phase
-      // is then k-2, whose parity equals k's, and a parity wait would pass.
-      if (!warp_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
-      if (!warp_wait(bar_full + 8 * s, ph, abort_flag, lim)) break;
+      const int s = it % SS, a = it % AS;
+      // First the A slot's previous contents must be consumed (its MMAs
+      // done).  That also settles the parity wait on the stage's full
+      // barrier: a group skips the other group's iterations and could
+      // otherwise reach round k of a stage while round k-1's copies are
+      // still in flight, when the barrier's last completed phase (k-2) has
+      // the parity of k.  MMA(it - AS) done implies every stage round
+      // before this one has landed, because AS <= SS.
+      if (!warp_wait(bar_afree + 8 * a, ((it / AS) & 1) ^ 1, abort_flag, lim)) break;
+      if (!warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
       tc_fence_after();
+      // all shared-memory reads first (independent), then the arithmetic,
+      // then one 32-column TMEM store of this row's 128 dequantized weights
       const uint32_t wbase = sbase + C::kOffW + s * kTileBytes;
+      uint4 v[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[c] = lds128(wbase + (c * kTileN + r) * 16);
       const uint32_t prm = lds32(wbase + kCodeBytes + 4 * r);
-      const uint32_t a_col = lane_base + C::kA0 + 32 * s;
+      uint32_t out[32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const uint32_t sh = (c < 2) ? 0 : 16;
         const uint32_t sc = (prm >> sh) & 0xFFu;
         const uint32_t a4 = ((prm >> (sh + 8)) & 0xFFu) * 0x01010101u;
-        const uint4 v = lds128(wbase + (c * kTileN + r) * 16);
-        uint32_t out[8];
-        dequant_chunk(v, sc, a4, out);
-        tmem_st_x8(a_col + 8 * c, out);
+        dequant_chunk(v[c], sc, a4, *reinterpret_cast<uint32_t(*)[8]>(out + 8 * c));
       }
+      tmem_st_x32(lane_base + C::kA0 + 32 * a, out);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dq + 8 * s);
+      if (lane == 0) mbar_arrive(bar_dq + 8 * a);
     }
 
     // -------------------------------------------------------- epilogue
     const int nthr = 128 * DQG;
-    pdl_wait();  // s_x, the workspace and Y belong to the preceding kernels' order
+    const int et = threadIdx.x - 64;  // epilogue thread index
+    pdl_wait();  // s_x and the outputs are ordered after the preceding kernel
     if (p.Y) {
-      const int et = threadIdx.x - 64;  // epilogue thread index
       for (int i = et; i < T; i += nthr)
         sx_s[i] = (m0 + i < p.M) ? p.s_x[m0 + i] : 0.0f;
     }
     warp_wait(bar_acc, 0, abort_flag, lim);
     tc_fence_after();
     // one thread turns the abort flag into a value every epilogue thread
-    // reads between the same two barriers, so the branch below is uniform
+    // reads between the same two barriers, so the branches below are uniform
     named_bar_sync(1, nthr);
     if (warp == 2 && lane == 0) {
       if (!hdr_ok) record_status(kDevBadPacked);
       *ep_flag = (*abort_flag || !hdr_ok) ? 0 : 1;
     }
+    __syncwarp();
     named_bar_sync(1, nthr);
     if (*ep_flag) {
       if (p.splits == 1) {
@@ -285,72 +325,89 @@ __global__ void __launch_bounds__(GemmCfg<T, STAGES, DQG>::kThreads, MINB)
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
               const int m = m0 + 16 * j + t;
-              if (m < p.M) {
-                const int32_t a = (int32_t)v[t];
-                if (p.Y) {
-                  const float y = (float)a * (sx_s[16 * j + t] * swn);
-                  p.Y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-                } else {
-                  p.acc[(size_t)m * p.N + n] = a;
-                }
-              }
+              if (m < p.M) store_out(p, m, n, (int32_t)v[t], sx_s[16 * j + t], swn);
             }
           }
         }
       } else {
-        // partials are token-major ([token][channel]) so that for each token
-        // a warp's 32 reductions hit one contiguous 128-byte line
-        int32_t* wtile = p.ws + (size_t)m_tile * T * p.n_pad + n;
+        // partial tile -> own shared memory, token-major: part[t][r]
+        // (the pipeline buffers are free: every copy landed and every MMA
+        // that read them completed)
+        int32_t* part = reinterpret_cast<int32_t*>(smem);
         for (int j = dg; j < T / 16; j += DQG) {
           uint32_t v[16];
           tmem_ld_x16(lane_base + 16 * j, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 16; ++t)
-            if (m0 + 16 * j + t < p.M)
-              red_add_s32(wtile + (size_t)(16 * j + t) * p.n_pad, (int32_t)v[t]);
-        }
-        __threadfence();
-        named_bar_sync(1, nthr);
-        uint32_t* cnt = p.counters + (size_t)m_tile * p.n_tiles + n_tile;
-        if (warp == 2 && lane == 0) {
-          const uint32_t old = atomicAdd(cnt, 1u);
-          *last_flag = (old == (uint32_t)(p.splits - 1)) ? 1 : 0;
-        }
-        named_bar_sync(1, nthr);
-        if (*last_flag) {
-          __threadfence();
-          for (int j = dg; j < T / 16; j += DQG) {
-            int32_t a[16];
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-              a[t] = (m0 + 16 * j + t < p.M) ? __ldcg(wtile + (size_t)(16 * j + t) * p.n_pad) : 0;
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-              const int m = m0 + 16 * j + t;
-              if (m < p.M) {
-                __stcg(wtile + (size_t)(16 * j + t) * p.n_pad, 0);
-                if (n < p.N) {
-                  if (p.Y) {
-                    const float y = (float)a[t] * (sx_s[16 * j + t] * swn);
-                    p.Y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-                  } else {
-                    p.acc[(size_t)m * p.N + n] = a[t];
-                  }
-                }
-              }
-            }
-          }
-          if (warp == 2 && lane == 0) *cnt = 0u;
+          for (int t = 0; t < 16; ++t) part[(16 * j + t) * kTileN + r] = (int32_t)v[t];
         }
       }
     }
+    __syncwarp();
+  }
+
+  if (p.splits > 1) {
+    // ------------------------------------ split-K reduction over the cluster
+    cluster_sync_all();  // every partial of the cluster is in shared memory
+    if (warp >= 2 && *ep_flag) {
+      const int nthr = 128 * DQG;
+      const int et = threadIdx.x - 64;
+      const int t_valid = min(T, p.M - m0);
+      const int total = t_valid * kTileN;
+      // slices of whole 16-byte groups (4 consecutive channels of a token)
+      const int per = ((total + p.splits - 1) / p.splits + 3) & ~3;
+      const int e0 = split * per, e1 = min(total, e0 + per);
+      const uint32_t part0 = sbase;
+      constexpr int kBatch = 2;  // groups in flight per thread and round
+      for (int eb = e0 + 4 * et; eb < e1; eb += 4 * nthr * kBatch) {
+        int4 acc4[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) acc4[b] = make_int4(0, 0, 0, 0);
+        // issue every remote load of the round before using any of them
+        for (int q = 0; q < p.splits; ++q) {
+          int4 got[kBatch];
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            const int e = eb + 4 * nthr * b;
+            got[b] = e < e1 ? dsmem_ld_v4(dsmem_map(part0 + 4u * (uint32_t)e, (uint32_t)q))
+                            : make_int4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            acc4[b].x += got[b].x;
+            acc4[b].y += got[b].y;
+            acc4[b].z += got[b].z;
+            acc4[b].w += got[b].w;
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          const int e = eb + 4 * nthr * b;
+          if (e >= e1) continue;
+          const int t = e / kTileN, r2 = e % kTileN;
+          const int n2 = n_tile * kTileN + r2;
+          // s_w is padded to whole channel blocks, so the 4-wide load is in bounds
+          const float4 sw4 = p.Y ? __ldg(reinterpret_cast<const float4*>(p.s_w + n2))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+          const int32_t av[4] = {acc4[b].x, acc4[b].y, acc4[b].z, acc4[b].w};
+          const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (n2 + i < p.N) store_out(p, m0 + t, n2 + i, av[i], sx_s[t], swv[i]);
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // no CTA leaves while another still reads its partials
   }
 
   // ------------------------------------------------------------ teardown
-  if (threadIdx.x == 0 && *abort_flag) {
-    // every MMA issued has completed before TMEM is released
-    mbar_wait(bar_acc, 0, nullptr, lim);
+  if (warp == 0) {
+    if (lane == 0 && *abort_flag) {
+      // every MMA issued has completed before TMEM is released
+      mbar_wait(bar_acc, 0, nullptr, lim);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -8,6 +8,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -85,58 +86,90 @@ struct Schedule {
   int T = 16, splits = 1, kt_per = 1, n_tiles = 1, m_tiles = 1, ctas = 1;
 };
 
+constexpr int kMaxSplits = 8;  // portable thread-block cluster size
+
+// Tokens per tile: the smallest MMA N (multiple of 16, up to 256) that
+// covers M, so decode shapes do no wasted MMA work beyond 16 tokens.
+int tile_tokens(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+
+// CTAs of one configuration that fit on an SM at once (shared memory and
+// TMEM permitting); matches the MINB column of the launch table below.
 int ctas_per_sm(int T) { return T <= 128 ? 2 : 1; }
 
+// Split-K factor from a wave model: CTAs run in waves of (SMs x CTAs per
+// SM); a wave costs the k tiles each CTA walks plus the latency to fill its
+// pipeline (in k-tile times: about 12 for the memory-bound small tiles, 9
+// for the compute-bound 256-token tile), and splitting adds the cluster
+// reduction, which grows with the partial tile (T / 16 column groups) and
+// the number of splits.  Ties go to more splits (more requests in flight).
+// W4A8_FORCE_SPLITS=<n> in the environment overrides the choice (tuning
+// experiments only).
 Schedule choose_schedule(int M, int N, int K, int sms) {
   Schedule s;
-  s.T = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  s.T = tile_tokens(M);
   s.n_tiles = (N + kTileN - 1) / kTileN;
   s.m_tiles = M > 0 ? (M + s.T - 1) / s.T : 0;
   const int kt = K / kTileK;
-  const int tiles = s.n_tiles * s.m_tiles;
-  int splits = 1;
-  if (tiles > 0 && tiles < sms) {
-    splits = (sms * ctas_per_sm(s.T)) / tiles;
-    if (splits < 1) splits = 1;
-    if (splits > kt) splits = kt;
+  const long tiles = (long)s.n_tiles * s.m_tiles;
+  const long slots = (long)sms * ctas_per_sm(s.T);
+  const double fill = s.T <= 64 ? 12.0 : s.T == 128 ? 10.0 : 9.0;
+  static const int forced = [] {
+    const char* e = getenv("W4A8_FORCE_SPLITS");
+    return e ? atoi(e) : 0;
+  }();
+  double best = 1e300;
+  for (int cand = 1; cand <= kMaxSplits && cand <= kt; ++cand) {
+    const int per = (kt + cand - 1) / cand;
+    const int eff = (kt + per - 1) / per;
+    if (eff != cand) continue;  // same schedule as a smaller candidate
+    const double waves = (double)((tiles * eff + slots - 1) / slots);
+    const double red = eff > 1 ? 2.0 + (s.T / 16) * eff / 8.0 : 0.0;
+    double cost = waves * (per + fill) + red;
+    if (forced > 0) cost = (eff == forced) ? 0.0 : 1.0 + cost;
+    if (cost <= best) {
+      best = cost;
+      s.splits = eff;
+      s.kt_per = per;
+    }
   }
-  s.kt_per = (kt + splits - 1) / splits;
-  s.splits = (kt + s.kt_per - 1) / s.kt_per;  // no empty split
-  s.ctas = tiles * s.splits;
+  s.ctas = (int)(tiles * s.splits);
   return s;
 }
 
-size_t workspace_bytes_for(const Schedule& s, int N) {
-  if (s.splits <= 1) return 0;
-  const size_t n_pad = (size_t)round_up(N, kTileN);
-  size_t partial = (size_t)s.m_tiles * n_pad * s.T * sizeof(int32_t);
-  partial = (partial + 255) / 256 * 256;
-  return partial + (size_t)s.m_tiles * s.n_tiles * sizeof(uint32_t);
-}
-
 // ------------------------------------------------------------- launches
-// Launch with or without programmatic dependent launch (PDL).
+// Launch with optional programmatic dependent launch (PDL) and cluster size.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                     bool pdl, Args&&... args) {
+                     bool pdl, int cluster_x, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
 }
 
-template <int T, int STAGES, int DQG, int MINB>
+template <int T, int SS, int AS, int DQG, int MINB>
 cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
                         cudaStream_t st, bool pdl) {
-  using C = GemmCfg<T, STAGES, DQG>;
-  auto k = w4a8_gemm_kernel<T, STAGES, DQG, MINB>;
+  using C = GemmCfg<T, SS, AS, DQG>;
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
@@ -145,12 +178,11 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_relaxed);
   }
-  return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, map, p);
+  return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, p.splits, map, p);
 }
 
 int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
-                int K, uint16_t* Y, int32_t* acc, void* workspace, size_t ws_bytes,
-                unsigned flags, void* stream) {
+                int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
   if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
   const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
   if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
@@ -163,9 +195,6 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   const int dev = current_device();
   if (dev < 0) return W4A8_ERR_CUDA;
   const Schedule s = choose_schedule(M, N, K, num_sms(dev));
-  const size_t need = workspace_bytes_for(s, N);
-  if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
-    return W4A8_ERR_WORKSPACE;
 
   const int n_pad = round_up(N, kTileN);
   const uint8_t* base = static_cast<const uint8_t*>(packed);
@@ -175,10 +204,6 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   p.s_x = s_x;
   p.Y = Y;
   p.acc = Y ? nullptr : acc;
-  p.ws = static_cast<int32_t*>(workspace);
-  size_t partial = need ? ((size_t)s.m_tiles * n_pad * s.T * 4 + 255) / 256 * 256 : 0;
-  p.counters = need ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + partial)
-                    : nullptr;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -190,17 +215,22 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   p.m_tiles = s.m_tiles;
   p.wait_limit_ns = kWaitLimitNs;
   p.hdr = reinterpret_cast<const PackedHeader*>(base);
+  // Only rows that exist are fetched when M < T: the MMA still reads T rows,
+  // but rows past M only feed accumulator columns that are never stored.
+  const int box_rows = M < s.T ? M : s.T;
+  p.x_tx_bytes = (uint32_t)box_rows * kTileK;
 
   CUtensorMap map;
-  if (!make_act_map(&map, Xq, M, K, s.T)) return W4A8_ERR_CUDA;
+  if (!make_act_map(&map, Xq, M, K, box_rows)) return W4A8_ERR_CUDA;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
   switch (s.T) {
-    case 16: e = launch_gemm<16, 6, 2, 2>(map, p, s.ctas, st, pdl); break;
-    case 32: e = launch_gemm<32, 6, 2, 2>(map, p, s.ctas, st, pdl); break;
-    case 64: e = launch_gemm<64, 6, 2, 2>(map, p, s.ctas, st, pdl); break;
-    case 128: e = launch_gemm<128, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
-    default: e = launch_gemm<256, 5, 2, 1>(map, p, s.ctas, st, pdl); break;
+    // (tokens, smem stages, TMEM A slots, dequant groups, CTAs per SM)
+    case 16: e = launch_gemm<16, 10, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
+    case 32: e = launch_gemm<32, 8, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
+    case 64: e = launch_gemm<64, 6, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
+    case 128: e = launch_gemm<128, 4, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
+    default: e = launch_gemm<256, 5, 4, 2, 1>(map, p, s.ctas, st, pdl); break;
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
@@ -229,7 +259,6 @@ const char* w4a8_status_string(int status) {
     case W4A8_ERR_INVALID_ARG: return "W4A8_ERR_INVALID_ARG";
     case W4A8_ERR_UNSUPPORTED_SHAPE: return "W4A8_ERR_UNSUPPORTED_SHAPE";
     case W4A8_ERR_MISALIGNED: return "W4A8_ERR_MISALIGNED";
-    case W4A8_ERR_WORKSPACE: return "W4A8_ERR_WORKSPACE";
     case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
     case W4A8_ERR_TIMEOUT: return "W4A8_ERR_TIMEOUT";
     case W4A8_ERR_BAD_PACKED: return "W4A8_ERR_BAD_PACKED";
@@ -296,38 +325,23 @@ int w4a8_quantize_act_ex(const float* X, int M, int K, int8_t* Xq, float* s_x, u
   if (!X || !Xq || !s_x) return W4A8_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(s_x, 4)) return W4A8_ERR_MISALIGNED;
   cudaError_t e = launch_k(act_quant_kernel, dim3(M), dim3(kActThreads), 0, as_stream(stream),
-                           (flags & W4A8_FLAG_PDL) != 0, X, M, K, Xq, s_x);
+                           (flags & W4A8_FLAG_PDL) != 0, 1, X, M, K, Xq, s_x);
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
-size_t w4a8_gemm_workspace_bytes(int M, int N, int K) {
-  if (M < 1 || N < 1 || K < 1 || K % kTileK != 0) return 0;
-  const int dev = current_device();
-  return workspace_bytes_for(choose_schedule(M, N, K, num_sms(dev < 0 ? 0 : dev)), N);
-}
-
-int w4a8_workspace_init(void* workspace, size_t bytes, void* stream) {
-  if (bytes == 0) return W4A8_OK;
-  if (!workspace) return W4A8_ERR_INVALID_ARG;
-  return cudaMemsetAsync(workspace, 0, bytes, as_stream(stream)) == cudaSuccess
-             ? W4A8_OK
-             : W4A8_ERR_CUDA;
-}
-
 int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M, int N, int K,
-              uint16_t* Y, void* workspace, size_t ws_bytes, void* stream) {
-  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, workspace, ws_bytes, 0u, stream);
+              uint16_t* Y, void* stream) {
+  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, 0u, stream);
 }
 
 int w4a8_gemm_ex(const int8_t* Xq, const float* s_x, const void* packed, int M, int N, int K,
-                 uint16_t* Y, void* workspace, size_t ws_bytes, unsigned flags, void* stream) {
-  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, workspace, ws_bytes, flags, stream);
+                 uint16_t* Y, unsigned flags, void* stream) {
+  return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, flags, stream);
 }
 
 int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K, int32_t* acc,
-                  void* workspace, size_t ws_bytes, void* stream) {
-  return gemm_common(Xq, nullptr, packed, M, N, K, nullptr, acc, workspace, ws_bytes, 0u,
-                     stream);
+                  void* stream) {
+  return gemm_common(Xq, nullptr, packed, M, N, K, nullptr, acc, 0u, stream);
 }
 
 int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits, int* ctas) {

@@ -18,7 +18,7 @@
  *     by an FP epilogue y = s_x[m] * s_w[n] * acc[m][n] stored as bf16.
  *
  * Conventions for every entry point:
- *   - Pointers named X, W, Xq, s_x, packed, Y, acc, workspace and the outputs
+ *   - Pointers named X, W, Xq, s_x, packed, Y, acc and the outputs
  *     of the unpack call are DEVICE pointers owned by the caller.  The library
  *     allocates no memory and never synchronizes the host, except in
  *     w4a8_get_status.  Work is enqueued on `stream` (a cudaStream_t passed as
@@ -55,7 +55,6 @@ typedef enum {
   W4A8_ERR_INVALID_ARG = -1,       /* NULL pointer, negative size, bad group */
   W4A8_ERR_UNSUPPORTED_SHAPE = -2, /* K % 128, K > 65536, N < 1 */
   W4A8_ERR_MISALIGNED = -3,        /* see the alignment rule above */
-  W4A8_ERR_WORKSPACE = -4,         /* workspace NULL or smaller than required */
   W4A8_ERR_CUDA = -5,              /* a CUDA runtime call failed */
   W4A8_ERR_TIMEOUT = -6,           /* a device-side bounded wait ran out */
   W4A8_ERR_BAD_PACKED = -7         /* packed buffer header does not match */
@@ -115,34 +114,20 @@ int w4a8_quantize_act(const float* X, int M, int K, int8_t* Xq, float* s_x,
                       void* stream);
 
 /*
- * Bytes of device workspace w4a8_gemm / w4a8_gemm_i32 need for this shape
- * (0 when the chosen schedule needs none).  The workspace holds INT32
- * split-K partial sums and arrival counters.  It must be zero-filled before
- * its first use (cudaMemset, or w4a8_workspace_init); every successful call
- * leaves it zero-filled again, so it can be reused by later calls on the
- * same stream without clearing.  After a call that reported an error,
- * initialize it again.  Two calls that may run at the same time on the GPU
- * must not share a workspace.
- */
-size_t w4a8_gemm_workspace_bytes(int M, int N, int K);
-
-/* Zero-fill a workspace of `bytes` bytes on `stream`. */
-int w4a8_workspace_init(void* workspace, size_t bytes, void* stream);
-
-/*
  * The W4A8 GEMM with the fused bf16 epilogue:
  *   Y[m][n] = bf16_rn( float(acc[m][n]) * (s_x[m] * s_w[n]) ),
  *   acc[m][n] = sum_k Xq[m][k] * (code[n][k] * s_u8 + a - 128)   (INT32)
  * with the weights dequantized in-kernel as (code * s_u8 + a) XOR 0x80
  * (key_machinery) and the products on tcgen05 INT8 tensor cores (lead).
- *   Xq [M][K] int8, s_x [M] float32, packed (from w4a8_quantize_weights),
- *   Y [M][N] bf16, workspace of w4a8_gemm_workspace_bytes(M, N, K) bytes.
+ *   Xq [M][K] int8, s_x [M] float32, packed (from w4a8_quantize_weights;
+ *   the caller must pass the N and K it was built for), Y [M][N] bf16.
  * The accumulator is exact; the epilogue differs from an exact FP64
- * evaluation by at most one bf16 ulp.
+ * evaluation by at most one bf16 ulp.  Shapes with few output tiles split K
+ * across a thread-block cluster of up to 8 CTAs whose partial sums are
+ * reduced on chip, so no scratch memory is needed.
  */
 int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M,
-              int N, int K, uint16_t* Y, void* workspace, size_t ws_bytes,
-              void* stream);
+              int N, int K, uint16_t* Y, void* stream);
 
 /*
  * Launch options for the *_ex entry points (bit mask).
@@ -158,8 +143,7 @@ int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M,
 
 /* w4a8_gemm with launch options (flags as above; 0 = w4a8_gemm). */
 int w4a8_gemm_ex(const int8_t* Xq, const float* s_x, const void* packed, int M,
-                 int N, int K, uint16_t* Y, void* workspace, size_t ws_bytes,
-                 unsigned flags, void* stream);
+                 int N, int K, uint16_t* Y, unsigned flags, void* stream);
 
 /* w4a8_quantize_act with launch options (flags as above).  With
  * W4A8_FLAG_PDL it waits for the preceding kernel before reading X. */
@@ -169,12 +153,12 @@ int w4a8_quantize_act_ex(const float* X, int M, int K, int8_t* Xq, float* s_x,
 /* Same product, writing the exact INT32 accumulators acc [M][N] instead of
  * the bf16 output (for bit-exact verification). */
 int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K,
-                  int32_t* acc, void* workspace, size_t ws_bytes,
-                  void* stream);
+                  int32_t* acc, void* stream);
 
 /*
  * Schedule the library picks for a shape (introspection for tests and
- * benchmarks): tokens per tile, split-K factor, number of CTAs.  Any output
+ * benchmarks): tokens per tile, split-K factor (= cluster size), number of
+ * CTAs.  Any output
  * pointer may be NULL.  Host-only.
  */
 int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,

@@ -33,7 +33,3 @@ def assert_bf16_within_1ulp(got_bits: np.ndarray, ref_bits: np.ndarray, what="")
     assert d.max(initial=0) <= 1, "%s: %d outputs off by more than 1 bf16 ulp, first at %s" % (
         what, bad[0].size, tuple(int(x[0]) for x in bad))
     return d
-
-
-def ws_is_zero(ws) -> bool:
-    return ws is None or int(ws.count_nonzero().item()) == 0

@@ -11,7 +11,7 @@ import torch
 import bit_block_quantized_w4a8_b200 as w4
 import oracle
 from bit_block_quantized_w4a8_b200 import workloads as wl
-from gpu_util import assert_bf16_within_1ulp, bf16_bits, require_gpu, ws_is_zero
+from gpu_util import assert_bf16_within_1ulp, bf16_bits, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -87,12 +87,11 @@ def _run_case(M, N, K, seed, wkind="normal", xkind="normal", group=64):
     acc_ref, y_ref = oracle.w4a8_gemm(Xq_ref, sx_ref, wq, group=group)
     pk = w4.w4a8_quantize_weights(W.cuda(), group=group)
     Xq, sx = w4.w4a8_quantize_act(X.cuda())
-    ws = w4.workspace_for(M, N, K)
-    acc = w4.w4a8_gemm_i32(Xq, pk, workspace=ws)
-    Y = w4.w4a8_gemm(Xq, sx, pk, workspace=ws)
+    acc = w4.w4a8_gemm_i32(Xq, pk)
+    Y = w4.w4a8_gemm(Xq, sx, pk)
     torch.cuda.synchronize()
     assert w4.w4a8_get_status() == 0
-    return acc.cpu().numpy(), bf16_bits(Y), acc_ref, y_ref, ws
+    return acc.cpu().numpy(), bf16_bits(Y), acc_ref, y_ref
 
 
 GEMM_SHAPES = [
@@ -113,23 +112,22 @@ GEMM_SHAPES = [
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
 def test_gemm_parity(M, N, K):
-    acc, y, acc_ref, y_ref, ws = _run_case(M, N, K, seed=M * 7 + N + K)
+    acc, y, acc_ref, y_ref = _run_case(M, N, K, seed=M * 7 + N + K)
     assert np.array_equal(acc, acc_ref)
     assert_bf16_within_1ulp(y, y_ref, "M=%d N=%d K=%d" % (M, N, K))
-    assert ws_is_zero(ws), "split-K workspace must be left zero-filled"
 
 
 @pytest.mark.parametrize("wkind,xkind", [("rowzero", "rowzero"), ("ties", "ties"),
                                          ("heavy", "heavy"), ("const", "const"),
                                          ("zeros", "normal"), ("normal", "zeros")])
 def test_gemm_parity_value_patterns(wkind, xkind):
-    acc, y, acc_ref, y_ref, _ = _run_case(40, 256, 512, seed=11, wkind=wkind, xkind=xkind)
+    acc, y, acc_ref, y_ref = _run_case(40, 256, 512, seed=11, wkind=wkind, xkind=xkind)
     assert np.array_equal(acc, acc_ref)
     assert_bf16_within_1ulp(y, y_ref)
 
 
 def test_gemm_parity_group128():
-    acc, y, acc_ref, y_ref, _ = _run_case(24, 256, 512, seed=12, group=128)
+    acc, y, acc_ref, y_ref = _run_case(24, 256, 512, seed=12, group=128)
     assert np.array_equal(acc, acc_ref)
     assert_bf16_within_1ulp(y, y_ref)
 
@@ -143,7 +141,7 @@ def test_gemm_int32_extremes():
     X[2, ::2] = -3.0
     W = torch.full((N, K), 0.5)
     W[:, 0] = -0.5
-    acc, y, acc_ref, y_ref, _ = _run_case_from(X, W)
+    acc, y, acc_ref, y_ref = _run_case_from(X, W)
     assert np.array_equal(acc, acc_ref)
     assert np.abs(acc_ref).max() > 100_000_000
     assert_bf16_within_1ulp(y, y_ref)
@@ -160,7 +158,7 @@ def _run_case_from(X, W, group=64):
     acc = w4.w4a8_gemm_i32(Xq, pk)
     Y = w4.w4a8_gemm(Xq, sx, pk)
     torch.cuda.synchronize()
-    return acc.cpu().numpy(), bf16_bits(Y), acc_ref, y_ref, None
+    return acc.cpu().numpy(), bf16_bits(Y), acc_ref, y_ref
 
 
 def test_gemm_deterministic_and_stream():
@@ -169,10 +167,10 @@ def test_gemm_deterministic_and_stream():
     pk = w4.w4a8_quantize_weights(W)
     Xq, sx = w4.w4a8_quantize_act(X)
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        ws = w4.workspace_for(5, 384, 1024, stream=s)
-        y1 = w4.w4a8_gemm(Xq, sx, pk, workspace=ws, stream=s)
-        y2 = w4.w4a8_gemm(Xq, sx, pk, workspace=ws, stream=s)
+        y1 = w4.w4a8_gemm(Xq, sx, pk, stream=s)
+        y2 = w4.w4a8_gemm(Xq, sx, pk, stream=s)
     s.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
@@ -195,16 +193,13 @@ def test_host_side_rejections():
     st = torch.cuda.current_stream().cuda_stream
     p = lambda t: t.data_ptr()
     # K not a multiple of 128
-    assert L.w4a8_gemm(p(Xq), p(sx), p(pk.data), 4, 128, 200, p(Y), None, 0, st) == w4.ERR_UNSUPPORTED_SHAPE
+    assert L.w4a8_gemm(p(Xq), p(sx), p(pk.data), 4, 128, 200, p(Y), st) == w4.ERR_UNSUPPORTED_SHAPE
     # misaligned activations
-    assert L.w4a8_gemm(p(Xq) + 1, p(sx), p(pk.data), 4, 128, 256, p(Y), None, 0, st) == w4.ERR_MISALIGNED
+    assert L.w4a8_gemm(p(Xq) + 1, p(sx), p(pk.data), 4, 128, 256, p(Y), st) == w4.ERR_MISALIGNED
     # missing output
-    assert L.w4a8_gemm(p(Xq), p(sx), p(pk.data), 4, 128, 256, None, None, 0, st) == w4.ERR_INVALID_ARG
-    # split-K shape without a workspace
-    Xq1 = torch.zeros(1, 4096, dtype=torch.int8, device="cuda")
-    Wb = w4.w4a8_quantize_weights(wl.random_matrix(128, 4096, 2, std=0.02).cuda())
-    assert w4.w4a8_gemm_workspace_bytes(1, 128, 4096) > 0
-    assert L.w4a8_gemm(p(Xq1), p(sx), p(Wb.data), 1, 128, 4096, p(Y), None, 0, st) == w4.ERR_WORKSPACE
+    assert L.w4a8_gemm(p(Xq), p(sx), p(pk.data), 4, 128, 256, None, st) == w4.ERR_INVALID_ARG
+    # unknown launch flag
+    assert L.w4a8_gemm_ex(p(Xq), p(sx), p(pk.data), 4, 128, 256, p(Y), 6, st) == w4.ERR_INVALID_ARG
     # bad group
     assert L.w4a8_quantize_weights(p(W), 128, 256, 32, p(pk.data), st) == w4.ERR_INVALID_ARG
     assert w4.w4a8_get_status() == 0
@@ -227,35 +222,32 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     w4.w4a8_debug_timeout_probe(2_000_000)  # 2 ms limit, nothing ever arrives
     assert w4.w4a8_get_status() == w4.ERR_TIMEOUT
     assert w4.w4a8_get_status() == 0
-    acc, y, acc_ref, y_ref, _ = _run_case(3, 128, 256, seed=5)
+    acc, y, acc_ref, y_ref = _run_case(3, 128, 256, seed=5)
     assert np.array_equal(acc, acc_ref)
 
 
 def test_pdl_chain_matches_plain_calls():
     """Chains of quantize -> GEMM launched with programmatic dependent launch
     (each kernel may start while the previous one finishes) give the same
-    bits as plain launches, including split-K shapes sharing one workspace."""
+    bits as plain launches, split-K (cluster) shapes included."""
     K = 2048
     W = wl.random_matrix(256, K, 41, std=0.02).cuda()
     pk = w4.w4a8_quantize_weights(W)
     Ms = [1, 3, 16, 40, 130, 300]
     Xs = [wl.random_matrix(M, K, 50 + M).cuda() for M in Ms]
-    ws = torch.zeros(max(w4.w4a8_gemm_workspace_bytes(M, 256, K) for M in Ms) + 256,
-                     dtype=torch.uint8, device="cuda")
     ref = []
     for X in Xs:
         xq, s = w4.w4a8_quantize_act(X)
-        ref.append(w4.w4a8_gemm(xq, s, pk, workspace=ws).clone())
+        ref.append(w4.w4a8_gemm(xq, s, pk).clone())
     for rep in range(3):
         outs = []
         for X in Xs:
             xq, s = w4.w4a8_quantize_act(X, flags=w4.W4A8_FLAG_PDL)
-            outs.append(w4.w4a8_gemm(xq, s, pk, workspace=ws, flags=w4.W4A8_FLAG_PDL))
+            outs.append(w4.w4a8_gemm(xq, s, pk, flags=w4.W4A8_FLAG_PDL))
         torch.cuda.synchronize()
         for a, b in zip(outs, ref):
             assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert w4.w4a8_get_status() == 0
-    assert ws_is_zero(ws)
 
 
 @pytest.mark.parametrize("M,N,K", [(512, 4096, 4096), (1024, 8192, 2048), (48, 2048, 8192)])
@@ -270,7 +262,6 @@ def test_repeated_runs_deep_k(M, N, K):
     W8 = oracle.dequant_weights(wq["codes"], wq["s_u8"], wq["a"])
     pk = w4.w4a8_quantize_weights(W.cuda())
     Xq, sx = w4.w4a8_quantize_act(X.cuda())
-    ws = w4.workspace_for(M, N, K)
     first = None
     rng = np.random.default_rng(M + N + K)
     ms = rng.integers(0, M, 256)
@@ -279,7 +270,7 @@ def test_repeated_runs_deep_k(M, N, K):
     row_ref = Xq_ref.astype(np.int64) @ W8.sum(axis=0, dtype=np.int64)
     col_ref = W8.astype(np.int64) @ Xq_ref.sum(axis=0, dtype=np.int64)
     for rep in range(6):
-        acc = w4.w4a8_gemm_i32(Xq, pk, workspace=ws)
+        acc = w4.w4a8_gemm_i32(Xq, pk)
         torch.cuda.synchronize()
         assert w4.w4a8_get_status() == 0
         if first is None:
@@ -289,4 +280,3 @@ def test_repeated_runs_deep_k(M, N, K):
             assert np.array_equal(acc.sum(dim=0, dtype=torch.int64).cpu().numpy(), col_ref)
         else:
             assert torch.equal(acc, first), "run %d differs from run 0" % rep
-    assert ws_is_zero(ws)
