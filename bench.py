@@ -499,15 +499,16 @@ def run_cuda(args):
 
 
 def run_profile_case(args):
-    """Small fixed case for profilers: pack the N=K=4096 layer once and run
-    one GEMM per requested M (no graphs, no timing)."""
+    """Small fixed case for profilers: pack one layer (default: the N=K=4096
+    decode layer; --profile-layer WORKLOAD:LAYER for another) and run one
+    GEMM per requested M (no graphs, no timing)."""
     import bit_block_quantized_w4a8_b200 as w4
     torch.cuda.set_device(0)
-    layer = wl.WORKLOADS[WORKLOAD].layers[0]
-    N, K = layer.N, layer.K
-    pk = w4.w4a8_quantize_weights(wl.layer_weights(WORKLOAD, layer).cuda())
+    name, lname = (args.profile_layer or WORKLOAD + ":square").split(":")
+    layer = [L for L in wl.WORKLOADS[name].layers if L.name == lname][0]
+    pk = w4.w4a8_quantize_weights(wl.layer_weights(name, layer).cuda())
     for M in [int(x) for x in args.profile.split(",")]:
-        Xq, sx = w4.w4a8_quantize_act(wl.layer_activations(WORKLOAD, layer, M).cuda())
+        Xq, sx = w4.w4a8_quantize_act(wl.layer_activations(name, layer, M).cuda())
         w4.w4a8_gemm(Xq, sx, pk)
     torch.cuda.synchronize()
     status = w4.w4a8_get_status()
@@ -602,6 +603,8 @@ def main(argv=None):
                     help="seconds of CPU work for the oracle baseline sample")
     ap.add_argument("--profile", default=None,
                     help="comma-separated Ms: run one GEMM each on N=K=4096 for a profiler")
+    ap.add_argument("--profile-layer", default=None, metavar="WORKLOAD:LAYER",
+                    help="layer for --profile (default decode_sweep_4096:square)")
     ap.add_argument("--all-configs", default=None, metavar="PATH",
                     help="time every workload case and write a JSON report to PATH")
     args = ap.parse_args(argv)
