@@ -77,7 +77,7 @@ struct GemmCfg {
   // shared memory: x tiles | w tiles | barriers | misc | s_x cache
   static constexpr int kOffW = SS * kXBytes;
   static constexpr int kOffBar = kOffW + SS * kTileBytes;
-  static constexpr int kNumBars = 2 * SS + 2 * AS + 1;
+  static constexpr int kNumBars = 2 * SS + 2 * AS + 2;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffSx = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffSx + 4 * T + 1024;  // + alignment slack
@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
   const uint32_t bar_dq = bar_empty + 8 * SS;       // + 8 as
   const uint32_t bar_afree = bar_dq + 8 * AS;       // + 8 as
   const uint32_t bar_acc = bar_afree + 8 * AS;
+  const uint32_t bar_done = bar_acc + 8;  // every epilogue warp finished with TMEM
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* ep_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
@@ -153,20 +154,27 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
   const int m0 = m_tile * T;
   const uint64_t lim = p.wait_limit_ns;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < SS; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+  // Every warp reaches a CTA-wide barrier converged: an aligned barrier
+  // reached by a warp in pieces (one lane late) can complete early and
+  // leave a phase open that a later barrier then completes without waiting.
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < SS; ++s) {
+        mbar_init(bar_full + 8 * s, 1);
+        mbar_init(bar_empty + 8 * s, 1);
+      }
+      for (int a = 0; a < AS; ++a) {
+        mbar_init(bar_dq + 8 * a, 4);
+        mbar_init(bar_afree + 8 * a, 1);
+      }
+      mbar_init(bar_acc, 1);
+      mbar_init(bar_done, 4 * DQG);
+      *abort_flag = 0;
+      fence_barrier_init();
+      pdl_launch_dependents();
     }
-    for (int a = 0; a < AS; ++a) {
-      mbar_init(bar_dq + 8 * a, 4);
-      mbar_init(bar_afree + 8 * a, 1);
-    }
-    mbar_init(bar_acc, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
+    __syncwarp();
+  } else if (warp == 1) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
     tmem_relinquish();
   }
@@ -174,7 +182,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -402,19 +409,21 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
   }
 
   // ------------------------------------------------------------ teardown
-  if (warp == 0) {
-    if (lane == 0 && *abort_flag) {
-      // every MMA issued has completed before TMEM is released
-      mbar_wait(bar_acc, 0, nullptr, lim);
-    }
+  // Each epilogue warp reports that it no longer touches TMEM; the warp that
+  // frees TMEM waits for all of them (and, after an abort, for every MMA).
+  if (warp >= 2) {
+    tc_fence_before();
     __syncwarp();
+    if (lane == 0) mbar_arrive(bar_done);
   }
-  tc_fence_before();
-  __syncthreads();
   if (warp == 1) {
+    warp_wait(bar_done, 0, nullptr, lim);
+    if (*abort_flag) warp_wait(bar_acc, 0, nullptr, lim);
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+  __syncwarp();
+  __syncthreads();
 }
 
 }  // namespace w4a8
