@@ -63,7 +63,7 @@ struct GemmParams {
   const PackedHeader* hdr;  // checked against (N, K) before any store
 };
 
-template <int T, int SS, int AS, int DQG>
+template <int T, int SS, int AS, int DQG, bool PUSH = false>
 struct GemmCfg {
   static_assert(T % 16 == 0 && T >= 16 && T <= 256, "MMA N for M=128");
   static_assert(AS <= SS, "the TMEM ring must not be deeper than the smem ring");
@@ -77,10 +77,18 @@ struct GemmCfg {
   // shared memory: x tiles | w tiles | barriers | misc | s_x cache
   static constexpr int kOffW = SS * kXBytes;
   static constexpr int kOffBar = kOffW + SS * kTileBytes;
-  static constexpr int kNumBars = 2 * SS + 2 * AS + 2;
+  static constexpr int kNumBars = 2 * SS + 2 * AS + 3;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffSx = kOffMisc + 16;
-  static constexpr int kSmemBytes = kOffSx + 4 * T + 1024;  // + alignment slack
+  // partial tiles of at most kPushMaxM tokens are pushed (remote atomic
+  // adds) into the cluster leader's receive buffer; larger ones are gathered
+  // from every CTA's stage buffers (remote atomics serialise at the leader)
+  static constexpr bool kPush = PUSH;
+  static constexpr int kPushMaxM = 8;
+  static_assert(!PUSH || T == 16, "push reduction is for the 16-token tile");
+  static constexpr int kOffRed = (kOffSx + 4 * T + 15) & ~15;
+  static constexpr int kRedBytes = kPush ? T * kTileN * 4 : 0;
+  static constexpr int kSmemBytes = kOffRed + kRedBytes + 1024;  // + alignment slack
   // the split-K partial tile reuses the pipeline buffers
   static_assert(T * kTileN * 4 <= kOffBar, "partial tile must fit the stage buffers");
 };
@@ -120,11 +128,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB>
-__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH>
+__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH>::kThreads, MINB)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const GemmParams p) {
-  using C = GemmCfg<T, SS, AS, DQG>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,6 +145,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
   const uint32_t bar_afree = bar_dq + 8 * AS;       // + 8 as
   const uint32_t bar_acc = bar_afree + 8 * AS;
   const uint32_t bar_done = bar_acc + 8;  // every epilogue warp finished with TMEM
+  const uint32_t bar_red = bar_done + 8;  // pushed partials landed (cluster leader)
+  const bool push = C::kPush && p.splits > 1 && p.M <= C::kPushMaxM;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* ep_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
@@ -169,6 +179,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
       }
       mbar_init(bar_acc, 1);
       mbar_init(bar_done, 4 * DQG);
+      mbar_init(bar_red, p.splits > 1 ? (uint32_t)(p.splits - 1) * 4 * DQG : 1u);
       *abort_flag = 0;
       fence_barrier_init();
       pdl_launch_dependents();
@@ -178,10 +189,18 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
     tmem_relinquish();
   }
+  if (push && split == 0) {  // the leader's receive buffer starts at zero
+    int4* red = reinterpret_cast<int4*>(smem + C::kOffRed);
+    for (int i = threadIdx.x; i < C::kRedBytes / 16; i += C::kThreads)
+      red[i] = make_int4(0, 0, 0, 0);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // every CTA of the cluster announces that its barriers and buffers are
+  // initialised; the matching wait comes just before the first remote access
+  if (push) cluster_arrive();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -336,7 +355,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
             }
           }
         }
-      } else {
+      } else if (!push) {
         // partial tile -> own shared memory, token-major: part[t][r]
         // (the pipeline buffers are free: every copy landed and every MMA
         // that read them completed)
@@ -350,11 +369,56 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
         }
       }
     }
+    if (push) {
+      // split-K by pushing: the other CTAs add their partials into the
+      // leader's receive buffer and arrive on its barrier; the leader adds
+      // its own partial and runs the epilogue
+      cluster_wait();
+      const int t_valid = min(T, p.M - m0);
+      const uint32_t red = sbase + C::kOffRed;
+      if (split != 0) {
+        if (*ep_flag) {
+          const uint32_t red0 = dsmem_map(red, 0);
+          for (int j = dg; j < T / 16; j += DQG) {
+            if (16 * j >= t_valid) break;
+            uint32_t v[16];
+            tmem_ld_x16(lane_base + 16 * j, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (16 * j + t < t_valid)
+                dsmem_red_add_s32(red0 + 4u * (uint32_t)((16 * j + t) * kTileN + r),
+                                  (int32_t)v[t]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(dsmem_map(bar_red, 0));  // also after an abort
+      } else {
+        warp_wait(bar_red, 0, abort_flag, lim);
+        if (*ep_flag) {
+          const int32_t* rb = reinterpret_cast<const int32_t*>(smem + C::kOffRed);
+          for (int j = dg; j < T / 16; j += DQG) {
+            if (16 * j >= t_valid) break;
+            uint32_t v[16];
+            tmem_ld_x16(lane_base + 16 * j, v);
+            tmem_wait_ld();
+            if (n < p.N) {
+#pragma unroll
+              for (int t = 0; t < 16; ++t) {
+                const int tt = 16 * j + t;
+                if (tt < t_valid)
+                  store_out(p, m0 + tt, n, (int32_t)v[t] + rb[tt * kTileN + r], sx_s[tt], swn);
+              }
+            }
+          }
+        }
+      }
+    }
     __syncwarp();
   }
 
-  if (p.splits > 1) {
-    // ------------------------------------ split-K reduction over the cluster
+  if (p.splits > 1 && !push) {
+    // ---------------------- split-K by gathering partials over the cluster
     cluster_sync_all();  // every partial of the cluster is in shared memory
     if (warp >= 2 && *ep_flag) {
       const int nthr = 128 * DQG;
@@ -416,6 +480,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG>::kThreads, MINB)
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_done);
   }
+  if (push && warp < 2) cluster_wait();  // pairs with the arrive at set-up
   if (warp == 1) {
     warp_wait(bar_done, 0, nullptr, lim);
     if (*abort_flag) warp_wait(bar_acc, 0, nullptr, lim);

@@ -165,11 +165,11 @@ cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB>
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false>
 cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
                         cudaStream_t st, bool pdl) {
-  using C = GemmCfg<T, SS, AS, DQG>;
-  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH>;
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
@@ -225,8 +225,15 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
   switch (s.T) {
-    // (tokens, smem stages, TMEM A slots, dequant groups, CTAs per SM)
-    case 16: e = launch_gemm<16, 10, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
+    // (tokens, smem stages, TMEM A slots, dequant groups, CTAs per SM[, push])
+    case 16:
+      // split decode with at most 8 tokens: push reduction (8 KB receive
+      // buffer, one stage fewer); otherwise the deeper ring
+      if (s.splits > 1 && M <= 8)
+        e = launch_gemm<16, 9, 4, 2, 2, true>(map, p, s.ctas, st, pdl);
+      else
+        e = launch_gemm<16, 10, 4, 2, 2>(map, p, s.ctas, st, pdl);
+      break;
     case 32: e = launch_gemm<32, 8, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
     case 64: e = launch_gemm<64, 6, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 4, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
