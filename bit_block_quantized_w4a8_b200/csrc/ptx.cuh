@@ -78,17 +78,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test with acquire at cluster scope: for barriers that other CTAs of
+// the cluster arrive on, so their shared::cluster writes are visible after.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // after `limit_ns` of global time or as soon as *abort is set by another
 // role of the CTA; on giving up it records kDevTimeout (once per device),
 // raises *abort so the other roles leave their loops too, and returns false.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int* abort,
                                           uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() {
+    return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (test()) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (test()) return true;
     if (abort && *abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       record_status(kDevTimeout);
