@@ -22,8 +22,7 @@ from .build import LIB as _LIB_PATH
 __all__ = [
     "W4A8Error", "lib", "w4a8_version", "w4a8_status_string",
     "w4a8_packed_weight_bytes", "w4a8_quantize_weights", "w4a8_unpack_weights",
-    "w4a8_quantize_act", "w4a8_gemm", "w4a8_gemm_fused", "w4a8_gemm_i32",
-    "w4a8_gemm_schedule",
+    "w4a8_quantize_act", "w4a8_gemm", "w4a8_gemm_i32", "w4a8_gemm_schedule",
     "w4a8_get_status", "w4a8_debug_timeout_probe", "PackedWeights",
 ]
 
@@ -72,7 +71,6 @@ def lib():
             "w4a8_quantize_act_ex": ([p, i32, i32, p, p, _ct.c_uint, p], i32),
             "w4a8_gemm_ex": ([p, p, p, i32, i32, i32, p, _ct.c_uint, p], i32),
             "w4a8_gemm": ([p, p, p, i32, i32, i32, p, p], i32),
-            "w4a8_gemm_fused": ([p, p, i32, i32, i32, p, p, p, _ct.c_uint, p], i32),
             "w4a8_gemm_i32": ([p, p, i32, i32, i32, p, p], i32),
             "w4a8_gemm_schedule": ([i32, i32, i32, p, p, p], i32),
             "w4a8_get_status": ([p], i32),
@@ -195,24 +193,6 @@ def w4a8_gemm(Xq, s_x, packed, out=None, stream=None, flags=0):
                              _stream(stream))
     _check(rc, "w4a8_gemm")
     return Y
-
-
-def w4a8_gemm_fused(X, packed, out=None, xq_out=None, sx_out=None, stream=None, flags=0):
-    """Activation quantization fused into the GEMM: returns (Y bf16 [M,N],
-    Xq int8 [M,K], s_x fp32 [M]), bit-identical to w4a8_quantize_act
-    followed by w4a8_gemm."""
-    _need(X, _torch.float32, 2, "X")
-    M, K = X.shape
-    if K != packed.K:
-        raise ValueError("X has K=%d, weights have K=%d" % (K, packed.K))
-    N = packed.N
-    dev = X.device
-    Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=dev)
-    Xq = xq_out if xq_out is not None else _torch.empty(M, K, dtype=_torch.int8, device=dev)
-    sx = sx_out if sx_out is not None else _torch.empty(M, dtype=_torch.float32, device=dev)
-    _check(lib().w4a8_gemm_fused(_ptr(X), _ptr(packed.data), M, N, K, _ptr(Y), _ptr(Xq),
-                                 _ptr(sx), int(flags), _stream(stream)), "w4a8_gemm_fused")
-    return Y, Xq, sx
 
 
 def w4a8_gemm_i32(Xq, packed, out=None, stream=None):

@@ -45,7 +45,6 @@
 #include <cstdint>
 #include "layout.cuh"
 #include "ptx.cuh"
-#include "quant.cuh"
 
 namespace w4a8 {
 
@@ -62,23 +61,14 @@ struct GemmParams {
   uint32_t x_tx_bytes;    // bytes of one activation box (rows * 128)
   unsigned long long wait_limit_ns;
   const PackedHeader* hdr;  // checked against (N, K) before any store
-  // fused activation quantization (FUSED kernels): fp32 X [M][K] in, and the
-  // INT8 codes / scales also written out by the channel-block-0 CTAs
-  const float* X;
-  int8_t* xq_out;
-  float* sx_out;
 };
 
-template <int T, int SS, int AS, int DQG, bool PUSH = false, bool FUSED = false>
+template <int T, int SS, int AS, int DQG, bool PUSH = false>
 struct GemmCfg {
   static_assert(T % 16 == 0 && T >= 16 && T <= 256, "MMA N for M=128");
   static_assert(AS <= SS, "the TMEM ring must not be deeper than the smem ring");
-  static_assert(!FUSED || T <= 32, "fused activation quantization is for decode tiles");
   static constexpr int kXBytes = T * kTileK;             // activation tile
-  static constexpr int kDqWarps = 4 * DQG;
-  static constexpr int kActWarps = FUSED ? 2 : 0;        // activation quantizers
-  static constexpr int kFirstActWarp = 2 + 4 * DQG;
-  static constexpr int kThreads = (2 + 4 * DQG + kActWarps) * 32;
+  static constexpr int kThreads = (2 + 4 * DQG) * 32;
   static constexpr int kA0 = T < 32 ? 32 : T;             // first A column
   static constexpr int kColsUsed = kA0 + 32 * AS;
   static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
@@ -87,7 +77,7 @@ struct GemmCfg {
   // shared memory: x tiles | w tiles | barriers | misc | s_x cache
   static constexpr int kOffW = SS * kXBytes;
   static constexpr int kOffBar = kOffW + SS * kTileBytes;
-  static constexpr int kNumBars = 2 * SS + 2 * AS + 4;
+  static constexpr int kNumBars = 2 * SS + 2 * AS + 3;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffSx = kOffMisc + 16;
   // partial tiles of at most kPushMaxM tokens are pushed (remote atomic
@@ -98,11 +88,7 @@ struct GemmCfg {
   static_assert(!PUSH || T == 16, "push reduction is for the 16-token tile");
   static constexpr int kOffRed = (kOffSx + 4 * T + 15) & ~15;
   static constexpr int kRedBytes = kPush ? T * kTileN * 4 : 0;
-  // fused: every cluster rank's partial absmax per token, then the two act
-  // warps' partials
-  static constexpr int kOffAmax = kOffRed + kRedBytes;
-  static constexpr int kAmaxBytes = FUSED ? (8 + 2) * T * 4 : 0;
-  static constexpr int kSmemBytes = kOffAmax + kAmaxBytes + 1024;  // + alignment slack
+  static constexpr int kSmemBytes = kOffRed + kRedBytes + 1024;  // + alignment slack
   // the split-K partial tile reuses the pipeline buffers
   static_assert(T * kTileN * 4 <= kOffBar, "partial tile must fit the stage buffers");
 };
@@ -143,11 +129,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool FUSED>
-__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads, MINB)
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH>
+__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH>::kThreads, MINB)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const GemmParams p) {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, FUSED>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,11 +147,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
   const uint32_t bar_acc = bar_afree + 8 * AS;
   const uint32_t bar_done = bar_acc + 8;  // every epilogue warp finished with TMEM
   const uint32_t bar_red = bar_done + 8;  // pushed partials landed (cluster leader)
-  const uint32_t bar_amax = bar_red + 8;  // fused: every rank's partial absmax landed
   const bool push = C::kPush && p.splits > 1 && p.M <= C::kPushMaxM;
-  // the cluster's split barrier (arrive at set-up, wait once later) is used
-  // whenever CTAs write into each other's shared memory
-  const bool cl_phase = push || (FUSED && p.splits > 1);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* ep_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
@@ -189,7 +171,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
   if (warp == 0) {
     if (lane == 0) {
       for (int s = 0; s < SS; ++s) {
-        mbar_init(bar_full + 8 * s, 1 + C::kActWarps);
+        mbar_init(bar_full + 8 * s, 1);
         mbar_init(bar_empty + 8 * s, 1);
       }
       for (int a = 0; a < AS; ++a) {
@@ -199,7 +181,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
       mbar_init(bar_acc, 1);
       mbar_init(bar_done, 4 * DQG);
       mbar_init(bar_red, p.splits > 1 ? (uint32_t)(p.splits - 1) * 4 * DQG : 1u);
-      mbar_init(bar_amax, (uint32_t)p.splits * 32 * (C::kActWarps ? C::kActWarps : 1));
       *abort_flag = 0;
       fence_barrier_init();
       pdl_launch_dependents();
@@ -219,9 +200,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // every CTA of the cluster announces that its barriers and buffers are
-  // initialised; each thread's matching wait comes once, before its first
-  // remote access (or at the end of its role)
-  if (cl_phase) cluster_arrive();
+  // initialised; the matching wait comes just before the first remote access
+  if (push) cluster_arrive();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -244,13 +224,11 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
                  kTileBytes, bar_full + 8 * it, pol);
       }
     }
-    if (!FUSED) {
-      pdl_wait();  // activations are produced by the preceding kernel
-      if (leader) {
-        for (int it = 0; it < pre; ++it)
-          tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
-                      bar_full + 8 * it);
-      }
+    pdl_wait();  // activations are produced by the preceding kernel
+    if (leader) {
+      for (int it = 0; it < pre; ++it)
+        tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
+                    bar_full + 8 * it);
     }
     issued = pre;
     __syncwarp();
@@ -262,9 +240,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
         mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         bulk_g2s(sbase + C::kOffW + s * kTileBytes, wsrc + (size_t)it * kTileBytes,
                  kTileBytes, bar_full + 8 * s, pol);
-        if (!FUSED)
-          tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
-                      bar_full + 8 * s);
+        tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
+                    bar_full + 8 * s);
       }
       __syncwarp();
       issued = it + 1;
@@ -275,7 +252,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
         mbar_wait(bar_full + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
     }
     __syncwarp();  // reconverge before any CTA- or cluster-wide barrier
-    if (cl_phase) cluster_wait();
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     // Whole warp waits, one elected lane issues the MMAs and commits.
@@ -300,8 +276,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
     }
     if (leader) tc_commit(bar_acc);  // also on abort: tracks every MMA issued
     __syncwarp();
-    if (cl_phase) cluster_wait();
-  } else if (warp < C::kFirstActWarp) {
+  } else {
     // --------------------------------------------- dequantization warps
     const int dg = (warp - 2) / 4;         // dequant group
     const int quarter = warp & 3;          // TMEM lane quarter of this warp
@@ -352,11 +327,10 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
     const int nthr = 128 * DQG;
     const int et = threadIdx.x - 64;  // epilogue thread index
     pdl_wait();  // s_x and the outputs are ordered after the preceding kernel
-    if (p.Y && !FUSED) {  // (fused: the activation warps computed sx_s)
+    if (p.Y) {
       for (int i = et; i < T; i += nthr)
         sx_s[i] = (m0 + i < p.M) ? p.s_x[m0 + i] : 0.0f;
     }
-    if (cl_phase) cluster_wait();
     warp_wait(bar_acc, 0, abort_flag, lim);
     tc_fence_after();
     // one thread turns the abort flag into a value every epilogue thread
@@ -400,6 +374,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
       // split-K by pushing: the other CTAs add their partials into the
       // leader's receive buffer and arrive on its barrier; the leader adds
       // its own partial and runs the epilogue
+      cluster_wait();
       const int t_valid = min(T, p.M - m0);
       const uint32_t red = sbase + C::kOffRed;
       if (split != 0) {
@@ -420,7 +395,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(dsmem_map(bar_red, 0));  // also after an abort
       } else {
-        warp_wait<true>(bar_red, 0, abort_flag, lim);
+        warp_wait<true>(bar_red, 0, abort_flag, lim);  // remote arrivals: cluster scope
         if (*ep_flag) {
           const int32_t* rb = reinterpret_cast<const int32_t*>(smem + C::kOffRed);
           for (int j = dg; j < T / 16; j += DQG) {
@@ -441,112 +416,12 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
       }
     }
     __syncwarp();
-  } else if (FUSED) {
-    // ----------------------------------- activation quantization (fused)
-    // The same arithmetic as act_quant_kernel: per token, absmax over the
-    // whole row, s_x = absmax / 127 (IEEE fp32 division), codes
-    // rint(x / s_x) clamped to +-127.  Each split CTA sees only its k range,
-    // so the partial absmax values are exchanged across the cluster first.
-    const int aw = warp - C::kFirstActWarp;  // 0 .. kActWarps-1
-    const int at = aw * 32 + lane;
-    constexpr int kAT = C::kActWarps * 32;
-    const int t_valid = min(T, p.M - m0);
-    const int k_lo = kt0 * kTileK, k_len = nk * kTileK;
-    float* amax_all = reinterpret_cast<float*>(smem + C::kOffAmax);  // [8][T]
-    float* amax_w = amax_all + 8 * T;                                // [2][T]
-    pdl_wait();  // X is produced by the preceding kernel
-    float mx[T];
-#pragma unroll
-    for (int t = 0; t < T; ++t) mx[t] = 0.0f;
-    for (int i = at; i < k_len / 4; i += kAT) {
-#pragma unroll
-      for (int t = 0; t < T; ++t)
-        if (t < t_valid) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(
-                                     p.X + (size_t)(m0 + t) * p.K + k_lo) + i);
-          mx[t] = fmaxf(mx[t], fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)),
-                                     fmaxf(fabsf(v.z), fabsf(v.w))));
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx[t] = fmaxf(mx[t], __shfl_xor_sync(0xffffffffu, mx[t], o));
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int t = 0; t < T; ++t) amax_w[aw * T + t] = mx[t];
-    }
-    named_bar_sync(2, kAT);
-    if (p.splits > 1) {
-      // publish this split's partial into every rank's table, then wait
-      // until every rank has published into ours
-      cluster_wait();
-      const uint32_t tab = sbase + C::kOffAmax;
-      for (int q = 0; q < p.splits; ++q) {
-        for (int t = at; t < t_valid; t += kAT) {
-          const float v = fmaxf(amax_w[t], amax_w[T + t]);
-          asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_map(
-                           tab + 4u * (uint32_t)(split * T + t), (uint32_t)q)),
-                       "f"(v)
-                       : "memory");
-        }
-        mbar_arrive_remote(dsmem_map(bar_amax, (uint32_t)q));
-      }
-      warp_wait<true>(bar_amax, 0, abort_flag, lim);
-      for (int t = at; t < T; t += kAT) {
-        float v = 0.0f;
-        if (t < t_valid)
-          for (int q = 0; q < p.splits; ++q) v = fmaxf(v, amax_all[q * T + t]);
-        sx_s[t] = __fdiv_rn(v, 127.0f);
-      }
-    } else {
-      for (int t = at; t < T; t += kAT)
-        sx_s[t] = t < t_valid ? __fdiv_rn(fmaxf(amax_w[t], amax_w[T + t]), 127.0f) : 0.0f;
-    }
-    named_bar_sync(2, kAT);
-    if (n_tile == 0 && split == 0 && p.sx_out)
-      for (int t = at; t < t_valid; t += kAT) p.sx_out[m0 + t] = sx_s[t];
-
-    // quantize the CTA's k range into the stage buffers, one k tile per
-    // stage, in the 128-byte-swizzled K-major layout the MMA descriptor
-    // describes (16-byte chunk j of row t at chunk j ^ (t % 8))
-    const bool write_xq = n_tile == 0 && p.xq_out != nullptr;
-    for (int it = 0; it < nk; ++it) {
-      const int s = it % SS;
-      const uint32_t ph = (it / SS) & 1;
-      if (!warp_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
-      const int k0 = (kt0 + it) * kTileK;
-      uint8_t* xt = smem + s * C::kXBytes;
-      for (int c = at; c < t_valid * 8; c += kAT) {
-        const int t = c >> 3, j = c & 7;
-        const float4* src = reinterpret_cast<const float4*>(p.X + (size_t)(m0 + t) * p.K + k0 + 16 * j);
-        const float sc = sx_s[t];
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 v = __ldg(src + q);
-          w[q] = (uint32_t)(quant_sym(v.x, sc, 127) & 0xFF) |
-                 ((uint32_t)(quant_sym(v.y, sc, 127) & 0xFF) << 8) |
-                 ((uint32_t)(quant_sym(v.z, sc, 127) & 0xFF) << 16) |
-                 ((uint32_t)(quant_sym(v.w, sc, 127) & 0xFF) << 24);
-        }
-        const uint4 packed4 = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(xt + t * 128 + ((j ^ (t & 7)) << 4)) = packed4;
-        if (write_xq)
-          *reinterpret_cast<uint4*>(p.xq_out + (size_t)(m0 + t) * p.K + k0 + 16 * j) = packed4;
-      }
-      fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_full + 8 * s);
-    }
-    __syncwarp();
   }
 
   if (p.splits > 1 && !push) {
     // ---------------------- split-K by gathering partials over the cluster
     cluster_sync_all();  // every partial of the cluster is in shared memory
-    if (warp >= 2 && warp < C::kFirstActWarp && *ep_flag) {
+    if (warp >= 2 && *ep_flag) {
       const int nthr = 128 * DQG;
       const int et = threadIdx.x - 64;
       const int t_valid = min(T, p.M - m0);
@@ -601,11 +476,12 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, FUSED>::kThreads
   // ------------------------------------------------------------ teardown
   // Each epilogue warp reports that it no longer touches TMEM; the warp that
   // frees TMEM waits for all of them (and, after an abort, for every MMA).
-  if (warp >= 2 && warp < C::kFirstActWarp) {
+  if (warp >= 2) {
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_done);
   }
+  if (push && warp < 2) cluster_wait();  // pairs with the arrive at set-up
   if (warp == 1) {
     warp_wait(bar_done, 0, nullptr, lim);
     if (*abort_flag) warp_wait(bar_acc, 0, nullptr, lim);

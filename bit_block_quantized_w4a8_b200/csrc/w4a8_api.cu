@@ -165,11 +165,11 @@ cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool FUSED = false>
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false>
 cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
                         cudaStream_t st, bool pdl) {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, FUSED>;
-  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, FUSED>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH>;
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
@@ -215,9 +215,6 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   p.m_tiles = s.m_tiles;
   p.wait_limit_ns = kWaitLimitNs;
   p.hdr = reinterpret_cast<const PackedHeader*>(base);
-  p.X = nullptr;
-  p.xq_out = nullptr;
-  p.sx_out = nullptr;
   // Only rows that exist are fetched when M < T: the MMA still reads T rows,
   // but rows past M only feed accumulator columns that are never stored.
   const int box_rows = M < s.T ? M : s.T;
@@ -241,69 +238,6 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     case 64: e = launch_gemm<64, 6, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 4, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
     default: e = launch_gemm<256, 5, 4, 2, 1>(map, p, s.ctas, st, pdl); break;
-  }
-  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
-}
-
-// Fused activation quantization + GEMM for decode tiles (T <= 32) when each
-// CTA's extra reads of fp32 X stay small; otherwise the quantizer kernel
-// followed by the GEMM.  Xq and s_x are outputs in both cases.
-constexpr long kFusedMaxXBytesPerCta = 64 * 1024;
-
-int gemm_fused(const float* X, const void* packed, int M, int N, int K, uint16_t* Y,
-               int8_t* Xq, float* s_x, unsigned flags, void* stream) {
-  if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
-  if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
-  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
-  if (M == 0) return W4A8_OK;
-  if (!X || !packed || !Y || !Xq || !s_x) return W4A8_ERR_INVALID_ARG;
-  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 2) || !aligned(Xq, 16) ||
-      !aligned(s_x, 4))
-    return W4A8_ERR_MISALIGNED;
-  const int dev = current_device();
-  if (dev < 0) return W4A8_ERR_CUDA;
-  const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
-  const Schedule s = choose_schedule(M, N, K, num_sms(dev));
-  const long x_bytes = (long)(M < s.T ? M : s.T) * s.kt_per * kTileK * 4;
-  if (s.T > 32 || x_bytes > kFusedMaxXBytesPerCta) {
-    const int rc = w4a8_quantize_act_ex(X, M, K, Xq, s_x, flags, stream);
-    if (rc != W4A8_OK) return rc;
-    return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, flags, stream);
-  }
-  const int n_pad = round_up(N, kTileN);
-  const uint8_t* base = static_cast<const uint8_t*>(packed);
-  GemmParams p;
-  p.tiles = base + tiles_offset_bytes(n_pad);
-  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
-  p.s_x = nullptr;
-  p.Y = Y;
-  p.acc = nullptr;
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.n_pad = n_pad;
-  p.kt_total = K / kTileK;
-  p.splits = s.splits;
-  p.kt_per_split = s.kt_per;
-  p.n_tiles = s.n_tiles;
-  p.m_tiles = s.m_tiles;
-  p.x_tx_bytes = 0;  // activations come from the CTA's own quantizer warps
-  p.wait_limit_ns = kWaitLimitNs;
-  p.hdr = reinterpret_cast<const PackedHeader*>(base);
-  p.X = X;
-  p.xq_out = Xq;
-  p.sx_out = s_x;
-  CUtensorMap map;  // unused by the fused kernels; passed for the signature
-  std::memset(&map, 0, sizeof(map));
-  cudaStream_t st = as_stream(stream);
-  cudaError_t e;
-  if (s.T == 16) {
-    if (s.splits > 1 && M <= 8)
-      e = launch_gemm<16, 9, 4, 2, 2, true, true>(map, p, s.ctas, st, pdl);
-    else
-      e = launch_gemm<16, 10, 4, 2, 2, false, true>(map, p, s.ctas, st, pdl);
-  } else {
-    e = launch_gemm<32, 8, 4, 2, 2, false, true>(map, p, s.ctas, st, pdl);
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
@@ -410,11 +344,6 @@ int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M, int
 int w4a8_gemm_ex(const int8_t* Xq, const float* s_x, const void* packed, int M, int N, int K,
                  uint16_t* Y, unsigned flags, void* stream) {
   return gemm_common(Xq, s_x, packed, M, N, K, Y, nullptr, flags, stream);
-}
-
-int w4a8_gemm_fused(const float* X, const void* packed, int M, int N, int K, uint16_t* Y,
-                    int8_t* Xq, float* s_x, unsigned flags, void* stream) {
-  return gemm_fused(X, packed, M, N, K, Y, Xq, s_x, flags, stream);
 }
 
 int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K, int32_t* acc,

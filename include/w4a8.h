@@ -150,23 +150,6 @@ int w4a8_gemm_ex(const int8_t* Xq, const float* s_x, const void* packed, int M,
 int w4a8_quantize_act_ex(const float* X, int M, int K, int8_t* Xq, float* s_x,
                          unsigned flags, void* stream);
 
-/*
- * Activation quantization fused into the GEMM (the step directly before the
- * product; review: supporting citation [29] for per-token INT8 activations):
- *   Y = w4a8_gemm(quantize_act(X)) with identical bits, and the INT8 codes
- *   and scales written to Xq [M][K] and s_x [M] (caller-owned outputs) as by
- *   w4a8_quantize_act.
- *   X [M][K] float32 (16-byte aligned), packed, Y [M][N] bf16, Xq, s_x.
- * For decode shapes (up to 32 tokens per tile, and at most 64 KB of fp32
- * activations per CTA) one kernel does both: each CTA quantizes the slice of
- * X it multiplies, exchanging per-token absmax partials across its split-K
- * cluster, while its packed weights are already streaming in.  Other shapes
- * run w4a8_quantize_act followed by w4a8_gemm.  flags as for w4a8_gemm_ex.
- */
-int w4a8_gemm_fused(const float* X, const void* packed, int M, int N, int K,
-                    uint16_t* Y, int8_t* Xq, float* s_x, unsigned flags,
-                    void* stream);
-
 /* Same product, writing the exact INT32 accumulators acc [M][N] instead of
  * the bf16 output (for bit-exact verification). */
 int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K,
