@@ -81,6 +81,22 @@ bool make_act_map(CUtensorMap* map, const int8_t* Xq, int M, int K, int rows) {
   return r == CUDA_SUCCESS;
 }
 
+// -------------------------------------------------- kernel attributes
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false>
+cudaError_t ensure_smem_attr() {
+  using C = GemmCfg<T, SS, AS, DQG, PUSH>;
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
+    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_relaxed);
+  }
+  return cudaSuccess;
+}
+
 // ------------------------------------------------------------ schedule
 struct Schedule {
   int T = 16, splits = 1, kt_per = 1, n_tiles = 1, m_tiles = 1, ctas = 1;
@@ -90,29 +106,65 @@ constexpr int kMaxSplits = 8;  // portable thread-block cluster size
 
 // Tokens per tile: the smallest MMA N (multiple of 16, up to 256) that
 // covers M, so decode shapes do no wasted MMA work beyond 16 tokens.
-int tile_tokens(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+// (Above 64 tokens the 256-token tile is used: one CTA per SM with a deeper
+// ring measured faster than two 128-token CTAs per SM.)
+int tile_tokens(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 256; }
+
+// 16-token tiles walking at most this many k tiles use the light ring
+// (three CTAs per SM).  W4A8_LIGHT16=0 in the environment turns it off
+// (tuning experiments only).
+constexpr int kLightMaxKt = 6;
+bool light16_enabled() {
+  static const bool ok = [] {
+    const char* v = getenv("W4A8_LIGHT16");
+    return !(v && v[0] == '0');
+  }();
+  return ok;
+}
 
 // CTAs of one configuration that fit on an SM at once (shared memory and
 // TMEM permitting); matches the MINB column of the launch table below.
-int ctas_per_sm(int T) { return T <= 128 ? 2 : 1; }
+int ctas_per_sm(int T, int kt_per) {
+  if (T == 16 && kt_per <= kLightMaxKt && light16_enabled()) return 3;
+  return T <= 128 ? 2 : 1;
+}
 
-// Split-K factor from a wave model: CTAs run in waves of (SMs x CTAs per
-// SM); a wave costs the k tiles each CTA walks plus the latency to fill its
-// pipeline (in k-tile times: about 12 for the memory-bound small tiles, 9
-// for the compute-bound 256-token tile), and splitting adds the cluster
-// reduction, which grows with the partial tile (T / 16 column groups) and
-// the number of splits.  Ties go to more splits (more requests in flight).
-// W4A8_FORCE_SPLITS=<n> in the environment overrides the choice (tuning
-// experiments only).
+// Split-K factor from a latency/bandwidth model of one launch, in
+// microseconds, calibrated on B200 against forced-split timings of the
+// decode and 7B/70B-like layer shapes:
+//   time = waves * (fill + kt_per * t_tile) + reduction
+// - a wave is as many clusters (the splits of one output tile) as the SMs
+//   hold at once; a cluster whose size is not a power of two does not tile
+//   the SMs of a GPC evenly, so only 92% of the slots count for it;
+// - fill is launch, pipeline fill and epilogue (3.5 us for 16..64-token
+//   tiles, 7.4 us for the 256-token tile);
+// - t_tile is one k tile's time per CTA: the slower of the CTA's own
+//   dequantize + MMA chain (0.27 us for 16 tokens, 0.29 us for 256) and its
+//   share of HBM bandwidth (8.7 KB of packed weights per CTA per k tile at
+//   6 TB/s sustained);
+// - the cluster reduction costs ~0.1 us per halving step plus, for the
+//   gather form, the partial tile (0.005 us per token column).
+// Ties go to more splits.  W4A8_FORCE_SPLITS=<n> and W4A8_FORCE_TILE=<tokens>
+// (not below the tile M needs) in the environment override the choice
+// (tuning only).
 Schedule choose_schedule(int M, int N, int K, int sms) {
   Schedule s;
   s.T = tile_tokens(M);
+  static const int forced_tile = [] {  // tuning experiments only
+    const char* e = getenv("W4A8_FORCE_TILE");
+    return e ? atoi(e) : 0;
+  }();
+  if (forced_tile == 16 || forced_tile == 32 || forced_tile == 64 || forced_tile == 128 ||
+      forced_tile == 256)
+    if (forced_tile >= s.T) s.T = forced_tile;
   s.n_tiles = (N + kTileN - 1) / kTileN;
   s.m_tiles = M > 0 ? (M + s.T - 1) / s.T : 0;
   const int kt = K / kTileK;
   const long tiles = (long)s.n_tiles * s.m_tiles;
-  const long slots = (long)sms * ctas_per_sm(s.T);
-  const double fill = s.T <= 64 ? 12.0 : s.T == 128 ? 10.0 : 9.0;
+  const double fill = s.T <= 64 ? (s.T == 16 ? 3.5 : 3.7) : s.T == 128 ? 6.0 : 7.4;
+  const double t_cta = s.T == 16 ? 0.27 : s.T == 32 ? 0.28 : s.T == 64 ? 0.32 : 0.29;
+  constexpr double kBytesPerUs = 6.0e6;  // sustained HBM read rate
+  const bool push = s.T == 16 && M <= GemmCfg<16, 9, 4, 2, true>::kPushMaxM;
   static const int forced = [] {
     const char* e = getenv("W4A8_FORCE_SPLITS");
     return e ? atoi(e) : 0;
@@ -122,10 +174,18 @@ Schedule choose_schedule(int M, int N, int K, int sms) {
     const int per = (kt + cand - 1) / cand;
     const int eff = (kt + per - 1) / per;
     if (eff != cand) continue;  // same schedule as a smaller candidate
-    const double waves = (double)((tiles * eff + slots - 1) / slots);
-    const double red = eff > 1 ? 2.0 + (s.T / 16) * eff / 8.0 : 0.0;
-    double cost = waves * (per + fill) + red;
-    if (forced > 0) cost = (eff == forced) ? 0.0 : 1.0 + cost;
+    const long slots = (long)sms * ctas_per_sm(s.T, per);
+    long per_wave = (eff & (eff - 1)) == 0 ? slots / eff : (long)(0.92 * slots / eff);
+    if (per_wave < 1) per_wave = 1;
+    const long waves = (tiles + per_wave - 1) / per_wave;
+    const long resident = (tiles < per_wave ? tiles : per_wave) * eff;
+    const double t_bw = resident * (double)kTileBytes / kBytesPerUs;
+    const double t_tile = t_cta > t_bw ? t_cta : t_bw;
+    const int lg = eff > 4 ? 3 : eff > 2 ? 2 : eff > 1 ? 1 : 0;
+    const double tok = M < s.T ? M : s.T;
+    const double red = lg * (0.1 + (push ? 0.05 : 0.005 * tok));
+    double cost = waves * (fill + per * t_tile) + red;
+    if (forced > 0) cost = (eff == forced) ? 0.0 : 1e6 + cost;
     if (cost <= best) {
       best = cost;
       s.splits = eff;
@@ -170,14 +230,8 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
                         cudaStream_t st, bool pdl) {
   using C = GemmCfg<T, SS, AS, DQG, PUSH>;
   auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH>;
-  static std::atomic<bool> attr_set[kMaxDevices];
-  const int dev = current_device();
-  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev].store(true, std::memory_order_relaxed);
-  }
+  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH>();
+  if (ea != cudaSuccess) return ea;
   return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, p.splits, map, p);
 }
 
@@ -226,17 +280,24 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   cudaError_t e;
   switch (s.T) {
     // (tokens, smem stages, TMEM A slots, dequant groups, CTAs per SM[, push])
-    case 16:
-      // split decode with at most 8 tokens: push reduction (8 KB receive
-      // buffer, one stage fewer); otherwise the deeper ring
-      if (s.splits > 1 && M <= 8)
-        e = launch_gemm<16, 9, 4, 2, 2, true>(map, p, s.ctas, st, pdl);
+    case 16: {
+      // Short k ranges (<= 6 tiles per CTA) use a light ring that fits three
+      // CTAs per SM, so a following launch's CTAs find room early and start
+      // fetching weights under programmatic dependent launch; long ones keep
+      // the deep ring.  Split decode with at most 8 tokens pushes partials
+      // (8 KB receive buffer).
+      const bool push = s.splits > 1 && M <= GemmCfg<16, 9, 4, 2, true>::kPushMaxM;
+      if (ctas_per_sm(16, s.kt_per) == 3)
+        e = push ? launch_gemm<16, 6, 3, 2, 3, true>(map, p, s.ctas, st, pdl)
+                 : launch_gemm<16, 6, 3, 2, 3>(map, p, s.ctas, st, pdl);
       else
-        e = launch_gemm<16, 10, 4, 2, 2>(map, p, s.ctas, st, pdl);
+        e = push ? launch_gemm<16, 9, 4, 2, 2, true>(map, p, s.ctas, st, pdl)
+                 : launch_gemm<16, 10, 4, 2, 2>(map, p, s.ctas, st, pdl);
       break;
+    }
     case 32: e = launch_gemm<32, 8, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
     case 64: e = launch_gemm<64, 6, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
-    case 128: e = launch_gemm<128, 4, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
+    case 128: e = launch_gemm<128, 4, 4, 2, 2>(map, p, s.ctas, st, pdl); break;  // tuning only
     default: e = launch_gemm<256, 5, 4, 2, 1>(map, p, s.ctas, st, pdl); break;
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
