@@ -593,6 +593,96 @@ def run_all_configs(args):
     return 0
 
 
+def run_compare(args):
+    """The pages' comparison points on one harness (each timed as a graph of
+    back-to-back calls over rotating weight copies larger than twice the L2):
+    this library's W4A8 GEMM with group 64 and group 128, its W8A8 kernel
+    (INT8 weights, same rings and epilogue, no dequantization), and two
+    library references -- cuBLASLt INT8 (torch._int_mm: INT32 output, no
+    epilogue; M padded to 32 rows where it needs more than 16) and cuBLAS
+    bf16 (torch.mm on unquantized weights).  Writes JSON to ``args.compare``."""
+    import bit_block_quantized_w4a8_b200 as w4
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    shapes = [("decode_sweep_4096", "square", [1, 4, 16, 64, 128, 256]),
+              ("llama7b_like", "qkv", [1, 16, 128, 1024]),
+              ("llama70b_like", "up", [1, 32, 512, 2048]),
+              ("llama70b_like", "down", [1, 32, 512, 2048])]
+    out = {"peaks": peaks, "cases": []}
+
+    def copies_of(t, nbytes):
+        n = max(1, min(32, -(-2 * l2 // nbytes)))
+        return [t] + [t.clone() for _ in range(n - 1)]
+
+    def timed(fn_i, n_in):
+        def body():
+            for i in range(n_in):
+                fn_i(i)
+        with torch.cuda.stream(stream):
+            fn_i(0)
+        stream.synchronize()
+        g = _graph(body, stream)
+        with torch.cuda.stream(stream):
+            g.replay()
+        reps = max(3, min(50, int(2e-3 / max(1e-6, _time_graph(g, 1, stream)))))
+        t = _time_graph(g, reps, stream) / n_in
+        del g
+        return t
+
+    for name, lname, Ms in shapes:
+        layer = [L for L in wl.WORKLOADS[name].layers if L.name == lname][0]
+        N, K = layer.N, layer.K
+        torch.cuda.empty_cache()
+        W = wl.layer_weights(name, layer).to(dev)
+        pk64 = w4.w4a8_quantize_weights(W, group=64)
+        pk128 = w4.w4a8_quantize_weights(W, group=128)
+        Wq, sw = w4.w8a8_quantize_weights(W)
+        Wbf = W.to(torch.bfloat16)
+        del W
+        c64 = copies_of(pk64.data, pk64.data.numel())
+        c128 = copies_of(pk128.data, pk128.data.numel())
+        c8 = copies_of(Wq, Wq.numel())
+        cbf = copies_of(Wbf, 2 * Wbf.numel())
+        p64 = [w4.PackedWeights(d, N, K, 64) for d in c64]
+        p128 = [w4.PackedWeights(d, N, K, 128) for d in c128]
+        for M in Ms:
+            X = wl.layer_activations(name, layer, M).to(dev)
+            Xq, sx = w4.w4a8_quantize_act(X)
+            Xbf = X.to(torch.bfloat16)
+            Mp = M if M > 16 else 32
+            Xq_p = torch.zeros(Mp, K, dtype=torch.int8, device=dev)
+            Xq_p[:M] = Xq
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            n_in = 8
+            t = {}
+            t["w4a8_g64"] = timed(lambda i: w4.w4a8_gemm(Xq, sx, p64[i % len(p64)], out=Y,
+                                                         stream=stream, flags=PDL), n_in)
+            t["w4a8_g128"] = timed(lambda i: w4.w4a8_gemm(Xq, sx, p128[i % len(p128)], out=Y,
+                                                          stream=stream, flags=PDL), n_in)
+            t["w8a8"] = timed(lambda i: w4.w8a8_gemm(Xq, sx, c8[i % len(c8)], sw, out=Y,
+                                                     stream=stream, flags=PDL), n_in)
+            t["cublaslt_int8_i32"] = timed(lambda i: torch._int_mm(Xq_p, c8[i % len(c8)].t()),
+                                           n_in)
+            t["cublas_bf16"] = timed(lambda i: torch.mm(Xbf, cbf[i % len(cbf)].t()), n_in)
+            status = w4.w4a8_get_status(stream)
+            o = gemm_ops(M, N, K)
+            case = {"workload": name, "layer": lname, "M": M, "N": N, "K": K, "status": status,
+                    "us": {k: v * 1e6 for k, v in t.items()},
+                    "tops": {k: o / v / 1e12 for k, v in t.items()},
+                    "w4a8_speedup": {k: v / t["w4a8_g64"] for k, v in t.items()},
+                    "m_padded_for_int_mm": Mp}
+            out["cases"].append(case)
+            print("%-18s %-6s M=%-5d " % (name, lname, M) + "  ".join(
+                "%s %.2fus" % (k, v * 1e6) for k, v in t.items()), flush=True)
+        del c64, c128, c8, cbf, p64, p128, pk64, pk128, Wq, sw, Wbf
+    with open(args.compare, "w") as f:
+        json.dump(out, f, indent=1)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -608,7 +698,12 @@ def main(argv=None):
                     help="layer for --profile (default decode_sweep_4096:square)")
     ap.add_argument("--all-configs", default=None, metavar="PATH",
                     help="time every workload case and write a JSON report to PATH")
+    ap.add_argument("--compare", default=None, metavar="PATH",
+                    help="time W4A8 (group 64/128), W8A8 and library GEMMs side by side; "
+                         "write a JSON report to PATH")
     args = ap.parse_args(argv)
+    if args.compare:
+        return run_compare(args)
     if args.all_configs:
         return run_all_configs(args)
     if args.profile:

@@ -24,6 +24,7 @@ __all__ = [
     "w4a8_packed_weight_bytes", "w4a8_quantize_weights", "w4a8_unpack_weights",
     "w4a8_quantize_act", "w4a8_gemm", "w4a8_gemm_i32", "w4a8_gemm_schedule",
     "w4a8_get_status", "w4a8_debug_timeout_probe", "PackedWeights",
+    "w8a8_quantize_weights", "w8a8_gemm", "w8a8_gemm_i32", "w8a8_gemm_schedule",
 ]
 
 OK = 0
@@ -73,6 +74,10 @@ def lib():
             "w4a8_gemm": ([p, p, p, i32, i32, i32, p, p], i32),
             "w4a8_gemm_i32": ([p, p, i32, i32, i32, p, p], i32),
             "w4a8_gemm_schedule": ([i32, i32, i32, p, p, p], i32),
+            "w8a8_quantize_weights": ([p, i32, i32, p, p, p], i32),
+            "w8a8_gemm": ([p, p, p, p, i32, i32, i32, p, _ct.c_uint, p], i32),
+            "w8a8_gemm_i32": ([p, p, i32, i32, i32, p, p], i32),
+            "w8a8_gemm_schedule": ([i32, i32, i32, p, p, p], i32),
             "w4a8_get_status": ([p], i32),
             "w4a8_debug_timeout_probe": ([ll, p], i32),
         }
@@ -213,6 +218,57 @@ def w4a8_gemm_schedule(M, N, K):
     t, s, c = _ct.c_int(0), _ct.c_int(0), _ct.c_int(0)
     _check(lib().w4a8_gemm_schedule(int(M), int(N), int(K), _ct.byref(t), _ct.byref(s),
                                     _ct.byref(c)), "w4a8_gemm_schedule")
+    return t.value, s.value, c.value
+
+
+def w8a8_quantize_weights(W, stream=None):
+    """Per-channel symmetric INT8 weights of fp32 W [N, K] for the W8A8
+    comparison kernel: returns (Wq int8 [N, K], s_w fp32 [N])."""
+    _need(W, _torch.float32, 2, "W")
+    N, K = W.shape
+    Wq = _torch.empty(N, K, dtype=_torch.int8, device=W.device)
+    sw = _torch.empty(N, dtype=_torch.float32, device=W.device)
+    _check(lib().w8a8_quantize_weights(_ptr(W), N, K, _ptr(Wq), _ptr(sw), _stream(stream)),
+           "w8a8_quantize_weights")
+    return Wq, sw
+
+
+def w8a8_gemm(Xq, s_x, Wq, s_w, out=None, stream=None, flags=0):
+    """W8A8 comparison GEMM: Y [M, N] bf16 = (s_x[m] s_w[n]) * sum_k Xq[m,k] Wq[n,k]."""
+    _need(Xq, _torch.int8, 2, "Xq")
+    _need(s_x, _torch.float32, 1, "s_x")
+    _need(Wq, _torch.int8, 2, "Wq")
+    _need(s_w, _torch.float32, 1, "s_w")
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s_w.numel() != N or s_x.numel() != M:
+        raise ValueError("shape mismatch: Xq %s, Wq %s, s_x %s, s_w %s"
+                         % (tuple(Xq.shape), tuple(Wq.shape), s_x.numel(), s_w.numel()))
+    Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
+    _check(lib().w8a8_gemm(_ptr(Xq), _ptr(s_x), _ptr(Wq), _ptr(s_w), M, N, K, _ptr(Y),
+                           int(flags), _stream(stream)), "w8a8_gemm")
+    return Y
+
+
+def w8a8_gemm_i32(Xq, Wq, out=None, stream=None):
+    """Exact INT32 accumulators of the W8A8 comparison GEMM."""
+    _need(Xq, _torch.int8, 2, "Xq")
+    _need(Wq, _torch.int8, 2, "Wq")
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("Xq has K=%d, Wq has K=%d" % (K, Wq.shape[1]))
+    acc = out if out is not None else _torch.empty(M, N, dtype=_torch.int32, device=Xq.device)
+    _check(lib().w8a8_gemm_i32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _stream(stream)),
+           "w8a8_gemm_i32")
+    return acc
+
+
+def w8a8_gemm_schedule(M, N, K):
+    """(tokens per tile, split-K factor, CTAs) of the W8A8 kernel for a shape."""
+    t, s, c = _ct.c_int(0), _ct.c_int(0), _ct.c_int(0)
+    _check(lib().w8a8_gemm_schedule(int(M), int(N), int(K), _ct.byref(t), _ct.byref(s),
+                                    _ct.byref(c)), "w8a8_gemm_schedule")
     return t.value, s.value, c.value
 
 

@@ -209,6 +209,20 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem,
       : "memory");
 }
 
+// D (TMEM) += A (shared memory, descriptor) x B (shared memory, descriptor).
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc,
+                                          uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0),
+      "r"(0), "r"(0)
+      : "memory");
+}
+
 // Each thread of the warp stores 8 consecutive 32-bit columns of its own
 // TMEM lane (lane = warp's lane quarter base + laneid).
 __device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&r)[8]) {

@@ -81,14 +81,31 @@ bool make_act_map(CUtensorMap* map, const int8_t* Xq, int M, int K, int rows) {
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over INT8 weights Wq [N][K] (K contiguous), for the W8A8
+// comparison kernel: boxes of 128 bytes of k by 128 channels, 128-byte
+// swizzle (the MMA's K-major operand layout), zero fill past channel N.
+bool make_w8_map(CUtensorMap* map, const int8_t* Wq, int N, int K) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)kTileN};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(Wq), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // -------------------------------------------------- kernel attributes
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false>
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false>
 cudaError_t ensure_smem_attr() {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
-    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH>,
+    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -123,9 +140,9 @@ bool light16_enabled() {
 }
 
 // CTAs of one configuration that fit on an SM at once (shared memory and
-// TMEM permitting); matches the MINB column of the launch table below.
-int ctas_per_sm(int T, int kt_per) {
-  if (T == 16 && kt_per <= kLightMaxKt && light16_enabled()) return 3;
+// TMEM permitting); matches the MINB column of the launch tables below.
+int ctas_per_sm(int T, int kt_per, bool w8) {
+  if (!w8 && T == 16 && kt_per <= kLightMaxKt && light16_enabled()) return 3;
   return T <= 128 ? 2 : 1;
 }
 
@@ -141,13 +158,15 @@ int ctas_per_sm(int T, int kt_per) {
 // - t_tile is one k tile's time per CTA: the slower of the CTA's own
 //   dequantize + MMA chain (0.27 us for 16 tokens, 0.29 us for 256) and its
 //   share of HBM bandwidth (8.7 KB of packed weights per CTA per k tile at
-//   6 TB/s sustained);
+//   6 TB/s sustained); the W8A8 comparison kernel reads 16 KB of weights
+//   per k tile through a shallower ring (bytes in flight per CTA bound it:
+//   0.35..0.45 us per k tile);
 // - the cluster reduction costs ~0.1 us per halving step plus, for the
 //   gather form, the partial tile (0.005 us per token column).
 // Ties go to more splits.  W4A8_FORCE_SPLITS=<n> and W4A8_FORCE_TILE=<tokens>
 // (not below the tile M needs) in the environment override the choice
 // (tuning only).
-Schedule choose_schedule(int M, int N, int K, int sms) {
+Schedule choose_schedule(int M, int N, int K, int sms, bool w8) {
   Schedule s;
   s.T = tile_tokens(M);
   static const int forced_tile = [] {  // tuning experiments only
@@ -162,7 +181,9 @@ Schedule choose_schedule(int M, int N, int K, int sms) {
   const int kt = K / kTileK;
   const long tiles = (long)s.n_tiles * s.m_tiles;
   const double fill = s.T <= 64 ? (s.T == 16 ? 3.5 : 3.7) : s.T == 128 ? 6.0 : 7.4;
-  const double t_cta = s.T == 16 ? 0.27 : s.T == 32 ? 0.28 : s.T == 64 ? 0.32 : 0.29;
+  const double t_cta = w8 ? (s.T == 16 ? 0.35 : s.T == 32 ? 0.40 : s.T == 64 ? 0.45 : 0.35)
+                         : (s.T > 64 ? 0.29 : s.T == 16 ? 0.27 : s.T == 32 ? 0.28 : 0.32);
+  const double w_bytes = w8 ? (double)kTileN * kTileK : (double)kTileBytes;
   constexpr double kBytesPerUs = 6.0e6;  // sustained HBM read rate
   const bool push = s.T == 16 && M <= GemmCfg<16, 9, 4, 2, true>::kPushMaxM;
   static const int forced = [] {
@@ -174,12 +195,12 @@ Schedule choose_schedule(int M, int N, int K, int sms) {
     const int per = (kt + cand - 1) / cand;
     const int eff = (kt + per - 1) / per;
     if (eff != cand) continue;  // same schedule as a smaller candidate
-    const long slots = (long)sms * ctas_per_sm(s.T, per);
+    const long slots = (long)sms * ctas_per_sm(s.T, per, w8);
     long per_wave = (eff & (eff - 1)) == 0 ? slots / eff : (long)(0.92 * slots / eff);
     if (per_wave < 1) per_wave = 1;
     const long waves = (tiles + per_wave - 1) / per_wave;
     const long resident = (tiles < per_wave ? tiles : per_wave) * eff;
-    const double t_bw = resident * (double)kTileBytes / kBytesPerUs;
+    const double t_bw = resident * w_bytes / kBytesPerUs;
     const double t_tile = t_cta > t_bw ? t_cta : t_bw;
     const int lg = eff > 4 ? 3 : eff > 2 ? 2 : eff > 1 ? 1 : 0;
     const double tok = M < s.T ? M : s.T;
@@ -225,57 +246,81 @@ cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false>
-cudaError_t launch_gemm(const CUtensorMap& map, const GemmParams& p, int ctas,
-                        cudaStream_t st, bool pdl) {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH>;
-  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH>;
-  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH>();
+// Tensor maps of one launch: activations, and the INT8 weights (W8A8 only;
+// a copy of the activation map stands in for the packed LQQ path).
+struct Maps {
+  CUtensorMap x, w;
+};
+
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false>
+cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream_t st,
+                        bool pdl) {
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8>;
+  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8>();
   if (ea != cudaSuccess) return ea;
-  return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, p.splits, map, p);
+  return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, p.splits, m.x,
+                  m.w, p);
 }
 
-int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
-                int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
+// Checks shared by both weight formats; fills the launch-independent part
+// of the parameters.  Returns W4A8_OK or an error (nothing launched).
+int check_common(const int8_t* Xq, const float* s_x, const void* w, int M, int N, int K,
+                 uint16_t* Y, int32_t* acc, unsigned flags) {
   if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
-  const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
   if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
   if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return W4A8_OK;
-  if (!Xq || !packed || (!Y && !acc) || (Y && !s_x)) return W4A8_ERR_INVALID_ARG;
-  if (!aligned(Xq, 16) || !aligned(packed, 16) || (Y && !aligned(Y, 2)) ||
+  if (!Xq || !w || (!Y && !acc) || (Y && !s_x)) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(w, 16) || (Y && !aligned(Y, 2)) ||
       (acc && !aligned(acc, 4)) || (s_x && !aligned(s_x, 4)))
     return W4A8_ERR_MISALIGNED;
-  const int dev = current_device();
-  if (dev < 0) return W4A8_ERR_CUDA;
-  const Schedule s = choose_schedule(M, N, K, num_sms(dev));
+  return W4A8_OK;
+}
 
-  const int n_pad = round_up(N, kTileN);
-  const uint8_t* base = static_cast<const uint8_t*>(packed);
+GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K, uint16_t* Y,
+                       int32_t* acc) {
   GemmParams p;
-  p.tiles = base + tiles_offset_bytes(n_pad);
-  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
+  p.tiles = nullptr;
+  p.s_w = nullptr;
   p.s_x = s_x;
   p.Y = Y;
   p.acc = Y ? nullptr : acc;
   p.M = M;
   p.N = N;
   p.K = K;
-  p.n_pad = n_pad;
+  p.n_pad = round_up(N, kTileN);
   p.kt_total = K / kTileK;
   p.splits = s.splits;
   p.kt_per_split = s.kt_per;
   p.n_tiles = s.n_tiles;
   p.m_tiles = s.m_tiles;
   p.wait_limit_ns = kWaitLimitNs;
-  p.hdr = reinterpret_cast<const PackedHeader*>(base);
+  p.hdr = nullptr;
   // Only rows that exist are fetched when M < T: the MMA still reads T rows,
   // but rows past M only feed accumulator columns that are never stored.
   const int box_rows = M < s.T ? M : s.T;
   p.x_tx_bytes = (uint32_t)box_rows * kTileK;
+  return p;
+}
 
-  CUtensorMap map;
-  if (!make_act_map(&map, Xq, M, K, box_rows)) return W4A8_ERR_CUDA;
+int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
+                int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
+  const int rc = check_common(Xq, s_x, packed, M, N, K, Y, acc, flags);
+  if (rc != W4A8_OK || M == 0) return rc;
+  const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
+  const int dev = current_device();
+  if (dev < 0) return W4A8_ERR_CUDA;
+  const Schedule s = choose_schedule(M, N, K, num_sms(dev), false);
+  GemmParams p = make_params(s, s_x, M, N, K, Y, acc);
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  p.tiles = base + tiles_offset_bytes(p.n_pad);
+  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
+  p.hdr = reinterpret_cast<const PackedHeader*>(base);
+
+  Maps m;
+  if (!make_act_map(&m.x, Xq, M, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
+  m.w = m.x;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
   switch (s.T) {
@@ -287,18 +332,56 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
       // the deep ring.  Split decode with at most 8 tokens pushes partials
       // (8 KB receive buffer).
       const bool push = s.splits > 1 && M <= GemmCfg<16, 9, 4, 2, true>::kPushMaxM;
-      if (ctas_per_sm(16, s.kt_per) == 3)
-        e = push ? launch_gemm<16, 6, 3, 2, 3, true>(map, p, s.ctas, st, pdl)
-                 : launch_gemm<16, 6, 3, 2, 3>(map, p, s.ctas, st, pdl);
+      if (ctas_per_sm(16, s.kt_per, false) == 3)
+        e = push ? launch_gemm<16, 6, 3, 2, 3, true>(m, p, s.ctas, st, pdl)
+                 : launch_gemm<16, 6, 3, 2, 3>(m, p, s.ctas, st, pdl);
       else
-        e = push ? launch_gemm<16, 9, 4, 2, 2, true>(map, p, s.ctas, st, pdl)
-                 : launch_gemm<16, 10, 4, 2, 2>(map, p, s.ctas, st, pdl);
+        e = push ? launch_gemm<16, 9, 4, 2, 2, true>(m, p, s.ctas, st, pdl)
+                 : launch_gemm<16, 10, 4, 2, 2>(m, p, s.ctas, st, pdl);
       break;
     }
-    case 32: e = launch_gemm<32, 8, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
-    case 64: e = launch_gemm<64, 6, 4, 2, 2>(map, p, s.ctas, st, pdl); break;
-    case 128: e = launch_gemm<128, 4, 4, 2, 2>(map, p, s.ctas, st, pdl); break;  // tuning only
-    default: e = launch_gemm<256, 5, 4, 2, 1>(map, p, s.ctas, st, pdl); break;
+    case 32: e = launch_gemm<32, 8, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
+    case 64: e = launch_gemm<64, 6, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
+    case 128: e = launch_gemm<128, 4, 4, 2, 2>(m, p, s.ctas, st, pdl); break;  // tuning only
+    default: e = launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl); break;
+  }
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+// The W8A8 comparison GEMM: the same kernel with plain INT8 weights read by
+// the MMA from shared memory (no dequantization warps: one group of four
+// epilogue warps).
+int gemm_w8_common(const int8_t* Xq, const float* s_x, const int8_t* Wq, const float* s_w,
+                   int M, int N, int K, uint16_t* Y, int32_t* acc, unsigned flags,
+                   void* stream) {
+  const int rc = check_common(Xq, s_x, Wq, M, N, K, Y, acc, flags);
+  if (rc != W4A8_OK || M == 0) return rc;
+  if (Y && !s_w) return W4A8_ERR_INVALID_ARG;
+  if (s_w && !aligned(s_w, 4)) return W4A8_ERR_MISALIGNED;
+  const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
+  const int dev = current_device();
+  if (dev < 0) return W4A8_ERR_CUDA;
+  const Schedule s = choose_schedule(M, N, K, num_sms(dev), true);
+  GemmParams p = make_params(s, s_x, M, N, K, Y, acc);
+  p.s_w = s_w;
+
+  Maps m;
+  if (!make_act_map(&m.x, Xq, M, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
+  if (!make_w8_map(&m.w, Wq, N, K)) return W4A8_ERR_CUDA;
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e;
+  switch (s.T) {
+    // (tokens, smem stages, -, epilogue groups, CTAs per SM, push, W8)
+    case 16: {
+      const bool push = s.splits > 1 && M <= GemmCfg<16, 5, 1, 1, true, true>::kPushMaxM;
+      e = push ? launch_gemm<16, 5, 1, 1, 2, true, true>(m, p, s.ctas, st, pdl)
+               : launch_gemm<16, 6, 1, 1, 2, false, true>(m, p, s.ctas, st, pdl);
+      break;
+    }
+    case 32: e = launch_gemm<32, 5, 1, 1, 2, false, true>(m, p, s.ctas, st, pdl); break;
+    case 64: e = launch_gemm<64, 4, 1, 1, 2, false, true>(m, p, s.ctas, st, pdl); break;
+    case 128: e = launch_gemm<128, 3, 1, 1, 2, false, true>(m, p, s.ctas, st, pdl); break;
+    default: e = launch_gemm<256, 4, 1, 1, 1, false, true>(m, p, s.ctas, st, pdl); break;
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
@@ -417,7 +500,36 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits, int* 
   if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
-  const Schedule s = choose_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev));
+  const Schedule s = choose_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev), false);
+  if (tile_tokens) *tile_tokens = s.T;
+  if (splits) *splits = s.splits;
+  if (ctas) *ctas = s.ctas;
+  return W4A8_OK;
+}
+
+int w8a8_quantize_weights(const float* W, int N, int K, int8_t* Wq, float* s_w, void* stream) {
+  // per-channel symmetric INT8: the per-row rule of the activation quantizer
+  if (N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  return w4a8_quantize_act_ex(W, N, K, Wq, s_w, 0u, stream);
+}
+
+int w8a8_gemm(const int8_t* Xq, const float* s_x, const int8_t* Wq, const float* s_w, int M,
+              int N, int K, uint16_t* Y, unsigned flags, void* stream) {
+  return gemm_w8_common(Xq, s_x, Wq, s_w, M, N, K, Y, nullptr, flags, stream);
+}
+
+int w8a8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32_t* acc,
+                  void* stream) {
+  return gemm_w8_common(Xq, nullptr, Wq, nullptr, M, N, K, nullptr, acc, 0u, stream);
+}
+
+int w8a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits, int* ctas) {
+  if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const Schedule s = choose_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev), true);
   if (tile_tokens) *tile_tokens = s.T;
   if (splits) *splits = s.splits;
   if (ctas) *ctas = s.ctas;

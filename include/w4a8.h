@@ -165,6 +165,42 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
                        int* ctas);
 
 /*
+ * ---- W8A8 comparison point ----
+ * The review page (pith summary; forward implication 3) measures the method
+ * against W8A8: 8-bit weights that need no dequantization.  These entry
+ * points run that product on the same kernel, rings, split-K reduction and
+ * epilogue, so that the two weight formats can be compared on one harness.
+ *
+ * Per-channel symmetric INT8 weights, by the same rule as the activations:
+ *   s_w[n] = max_k |W[n][k]| / 127 (fp32 division),
+ *   Wq[n][k] = clamp(rint(W[n][k] / s_w[n]), -127, 127), ties to even;
+ *   an all-zero channel gives s_w = 0 and Wq = 0.
+ *   W [N][K] float32 -> Wq [N][K] int8 (row-major, 16-byte aligned),
+ *   s_w [N] float32 (device, caller-owned).  K must be a multiple of 128.
+ */
+int w8a8_quantize_weights(const float* W, int N, int K, int8_t* Wq, float* s_w,
+                          void* stream);
+
+/*
+ * Y[m][n] = bf16_rn( float(acc[m][n]) * (s_x[m] * s_w[n]) ),
+ * acc[m][n] = sum_k Xq[m][k] * Wq[n][k]   (INT32, exact).
+ *   Xq [M][K] int8, s_x [M] float32, Wq [N][K] int8, s_w [N] float32,
+ *   Y [M][N] bf16 (all device, caller-owned; Xq and Wq 16-byte aligned).
+ * flags: W4A8_FLAG_PDL or 0.  Same shape rules and error codes as w4a8_gemm.
+ */
+int w8a8_gemm(const int8_t* Xq, const float* s_x, const int8_t* Wq,
+              const float* s_w, int M, int N, int K, uint16_t* Y,
+              unsigned flags, void* stream);
+
+/* The W8A8 product's exact INT32 accumulators acc [M][N]. */
+int w8a8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
+                  int32_t* acc, void* stream);
+
+/* Schedule of the W8A8 kernel for a shape (as w4a8_gemm_schedule). */
+int w8a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
+                       int* ctas);
+
+/*
  * Waits for `stream`, then returns and clears the device status word of the
  * current device: W4A8_OK, or W4A8_ERR_TIMEOUT if a kernel's bounded wait
  * ran out since the last call.  W4A8_ERR_CUDA if the synchronization failed.

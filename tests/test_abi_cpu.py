@@ -81,6 +81,14 @@ def test_argument_checks_before_any_launch(L):
     assert L.w4a8_quantize_weights(None, 128, 256, 64, None, st) == w4.ERR_INVALID_ARG
     assert L.w4a8_unpack_weights(None, 128, 256, None, None, None, None, st) == w4.ERR_INVALID_ARG
     assert L.w4a8_debug_timeout_probe(10, st) == w4.ERR_INVALID_ARG
+    # the W8A8 comparison entry points follow the same rules
+    assert L.w8a8_gemm(None, None, None, None, 4, 128, 200, None, 0, st) == w4.ERR_UNSUPPORTED_SHAPE
+    assert L.w8a8_gemm(None, None, None, None, 0, 128, 256, None, 0, st) == w4.OK
+    assert L.w8a8_gemm(None, None, None, None, 0, 128, 256, None, 4, st) == w4.ERR_INVALID_ARG
+    assert L.w8a8_gemm(None, None, None, None, 4, 128, 256, None, 0, st) == w4.ERR_INVALID_ARG
+    assert L.w8a8_gemm_i32(None, None, 0, 128, 256, None, st) == w4.OK
+    assert L.w8a8_quantize_weights(None, 128, 200, None, None, st) == w4.ERR_UNSUPPORTED_SHAPE
+    assert L.w8a8_quantize_weights(None, 0, 256, None, None, st) == w4.ERR_INVALID_ARG
 
 
 def test_schedule_covers_the_machine(L):
@@ -99,3 +107,14 @@ def test_schedule_covers_the_machine(L):
             assert -(-kt // per) == splits             # no empty split
             n_tiles, m_tiles = -(-N // 128), -(-M // T)
             assert ctas == n_tiles * m_tiles * splits
+
+
+def test_w8a8_schedule_covers_the_machine(L):
+    for M in (1, 8, 16, 17, 64, 65, 256, 4096):
+        for N, K in ((4096, 4096), (28672, 8192), (8192, 28672)):
+            T, splits, ctas = w4.w8a8_gemm_schedule(M, N, K)
+            assert T >= min(M, 16) and 1 <= splits <= 8
+            kt = K // 128
+            per = -(-kt // splits)
+            assert -(-kt // per) == splits
+            assert ctas == -(-N // 128) * -(-M // T) * splits

@@ -302,3 +302,56 @@ def test_epilogue_scales_and_signs():
     Y = oracle.bf16_bits_to_float(oracle.epilogue_bf16(acc, s_x, s_w))
     ref = (s_x[:, None].astype(np.float64) * s_w[None] * acc).astype(np.float32)
     assert np.array_equal(Y, torch.from_numpy(ref).to(torch.bfloat16).float().numpy())
+
+
+# ------------------------------------------- W8A8 comparison point (F2)
+
+def test_w8a8_weight_quant_hand_cases():
+    """Per-channel symmetric INT8 (the activations' per-row rule applied to
+    weight rows), on exactly representable values worked out by hand."""
+    W = np.array([[127.0, -63.5, 31.75, 0.5, 0.0, -1.5, 2.5, 0.0],
+                  [0.0] * 8,
+                  [2.5, -254.0, 1.0, 3.0, -3.0, 0.0, 5.0, 127.0]], np.float32)
+    Wq, s_w = oracle.w8a8_quantize_weights(W)
+    assert s_w.tolist() == [1.0, 0.0, 2.0]
+    # ties go to even: -63.5 -> -64, 0.5 -> 0, -1.5 -> -2, 2.5 -> 2
+    assert Wq[0].tolist() == [127, -64, 32, 0, 0, -2, 2, 0]
+    assert Wq[1].tolist() == [0] * 8
+    # row 2 divided by 2: 1.25, -127, 0.5, 1.5, -1.5, 0, 2.5, 63.5
+    assert Wq[2].tolist() == [1, -127, 0, 2, -2, 0, 2, 64]
+
+
+def test_w8a8_oracle_equals_w4a8_oracle_on_lqq_weights():
+    """Fed the dequantized LQQ weights as its INT8 operand (with the same
+    per-channel scales), the W8A8 product must reproduce the W4A8 product
+    bit for bit: both are sum_k Xq[m,k] W8[n,k] then the same epilogue, so a
+    transposed operand or a swapped scale in either one fails here."""
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((7, 320)).astype(np.float32)
+    W = (rng.standard_normal((52, 320)) * 0.02).astype(np.float32)
+    Xq, s_x = oracle.quantize_act(X)
+    wq = oracle.quantize_weights(W)
+    W8 = oracle.dequant_weights(wq["codes"], wq["s_u8"], wq["a"])
+    acc4, y4 = oracle.w4a8_gemm(Xq, s_x, wq)
+    acc8, y8 = oracle.w8a8_gemm(Xq, s_x, W8, wq["s_w"])
+    assert np.array_equal(acc4, acc8) and np.array_equal(y4, y8)
+    ms = np.array([0, 6, 3]); ns = np.array([51, 0, 17])
+    a2, y2 = oracle.w8a8_gemm_sampled(Xq, s_x, W8, wq["s_w"], ms, ns)
+    assert np.array_equal(a2, acc8[ms, ns]) and np.array_equal(y2, y8[ms, ns])
+
+
+def test_w8a8_error_bound_against_unquantized_product():
+    """|Y - X W^T| is within the quantization error bound |X| (s_w/2)
+    + (s_x/2) |W_hat| plus one bf16 rounding."""
+    rng = np.random.default_rng(9)
+    X = rng.standard_normal((9, 256)).astype(np.float32)
+    W = (rng.standard_normal((33, 256)) * 0.02).astype(np.float32)
+    Xq, s_x = oracle.quantize_act(X)
+    Wq, s_w = oracle.w8a8_quantize_weights(W)
+    _, Y = oracle.w8a8_gemm(Xq, s_x, Wq, s_w)
+    Yf = oracle.bf16_bits_to_float(Y).astype(np.float64)
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    What = Wq * s_w[:, None].astype(np.float64)
+    bound = np.abs(X) @ np.broadcast_to(s_w[:, None] / 2.0, W.shape).T \
+        + np.broadcast_to(s_x[:, None] / 2.0, X.shape) @ np.abs(What).T
+    assert np.all(np.abs(Yf - ref) <= bound * (1 + 1e-9) + np.abs(Yf) * 2.0 ** -8)
