@@ -683,6 +683,98 @@ def run_compare(args):
     return 0
 
 
+def run_moe(args):
+    """The grouped (mixture-of-experts) GEMM on the Mixtral-like expert layers
+    (8 experts, top-2): one grouped launch per layer call, against one dense
+    launch per expert that has rows.  Both timed as graphs of back-to-back
+    calls (programmatic dependent launch) over rotating copies of the expert
+    weights, with at least twice the L2 of active expert bytes.  Writes JSON
+    to ``args.moe``."""
+    import bit_block_quantized_w4a8_b200 as w4
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    name = "mixtral_like"
+    w = wl.MOE_WORKLOADS[name]
+    out = {"peaks": peaks, "workload": name, "cases": []}
+    for layer in w.layers:
+        N, K = layer.N, layer.K
+        b = w4.w4a8_packed_weight_bytes(N, K)
+        torch.cuda.empty_cache()
+        data = torch.empty(w.experts * b, dtype=torch.uint8, device=dev)
+        for e in range(w.experts):
+            w4.w4a8_quantize_weights(wl.moe_expert_weights(name, layer, e).to(dev),
+                                     out=data[e * b:(e + 1) * b])
+        for tokens in w.tokens:
+            offsets, tok = wl.moe_routing(name, tokens)
+            o = offsets.tolist()
+            active = [e for e in range(w.experts) if o[e + 1] > o[e]]
+            act_bytes = len(active) * weight_bytes(N, K)
+            ncopy = max(1, min(4, -(-2 * l2 // act_bytes)))
+            copies = [data] + [data.clone() for _ in range(ncopy - 1)]
+            gws = [w4.GroupedPackedWeights(d, w.experts, N, K, GROUP) for d in copies]
+            X = wl.moe_activations(name, layer, tokens)[tok].contiguous().to(dev)
+            M = X.shape[0]
+            Xq, sx = w4.w4a8_quantize_act(X)
+            off = offsets.to(dev)
+            mr = max(o[e + 1] - o[e] for e in range(w.experts))
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            n_in = 8
+
+            def grouped():
+                for i in range(n_in):
+                    w4.w4a8_grouped_gemm(Xq, sx, gws[i % ncopy], off, max_rows=mr, out=Y,
+                                         stream=stream, flags=PDL)
+
+            views = [(o[e], o[e + 1], [g.expert(e) for g in gws]) for e in active]
+
+            def per_expert():
+                for i in range(n_in):
+                    for r0, r1, ex in views:
+                        w4.w4a8_gemm(Xq[r0:r1], sx[r0:r1], ex[i % ncopy], out=Y[r0:r1],
+                                     stream=stream, flags=PDL)
+            t = {}
+            for key, fn in (("grouped", grouped), ("per_expert_dense", per_expert)):
+                with torch.cuda.stream(stream):
+                    fn()
+                stream.synchronize()
+                g = _graph(fn, stream)
+                with torch.cuda.stream(stream):
+                    g.replay()
+                reps = max(3, min(50, int(2e-3 / max(1e-6, _time_graph(g, 1, stream)))))
+                t[key] = _time_graph(g, reps, stream) / n_in
+                del g
+            status = w4.w4a8_get_status(stream)
+            ops = 2.0 * M * N * K
+            tot_bytes = act_bytes + M * K + 4 * M + 2 * M * N
+            hbm_t, tc_t = tot_bytes / (peaks["hbm"] * 1e9), ops / (peaks["bf16"] * INT8_PER_BF16 * 1e12)
+            bound = "hbm" if hbm_t >= tc_t else "tensor"
+            tg = t["grouped"]
+            T, splits, ctas = w4.w4a8_grouped_gemm_schedule(w.experts, M, mr, N, K)
+            case = {"layer": layer.name, "tokens": tokens, "rows": M, "N": N, "K": K,
+                    "active_experts": len(active), "max_rows": mr, "status": status,
+                    "grouped_us": tg * 1e6, "per_expert_dense_us": t["per_expert_dense"] * 1e6,
+                    "speedup_vs_per_expert": t["per_expert_dense"] / tg,
+                    "active_weight_gbs": act_bytes / tg / 1e9, "tops": ops / tg / 1e12,
+                    "bound": bound, "frac": (hbm_t if bound == "hbm" else tc_t) / tg,
+                    "schedule": {"tile_tokens": T, "splits": splits, "ctas": ctas},
+                    "weight_copies": ncopy}
+            out["cases"].append(case)
+            print("%-8s tokens=%-4d rows=%-5d experts=%d grouped %8.2f us  per-expert %8.2f us  "
+                  "x%.2f  %7.0f wGB/s %7.1f TOPS %-6s %.3f %s" % (
+                      layer.name, tokens, M, len(active), tg * 1e6,
+                      t["per_expert_dense"] * 1e6, case["speedup_vs_per_expert"],
+                      case["active_weight_gbs"], case["tops"], bound, case["frac"],
+                      case["schedule"]), flush=True)
+            del copies, gws
+        del data
+    with open(args.moe, "w") as f:
+        json.dump(out, f, indent=1)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -701,7 +793,12 @@ def main(argv=None):
     ap.add_argument("--compare", default=None, metavar="PATH",
                     help="time W4A8 (group 64/128), W8A8 and library GEMMs side by side; "
                          "write a JSON report to PATH")
+    ap.add_argument("--moe", default=None, metavar="PATH",
+                    help="time the grouped (mixture-of-experts) GEMM on the Mixtral-like "
+                         "layers; write a JSON report to PATH")
     args = ap.parse_args(argv)
+    if args.moe:
+        return run_moe(args)
     if args.compare:
         return run_compare(args)
     if args.all_configs:

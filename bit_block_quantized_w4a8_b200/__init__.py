@@ -25,6 +25,8 @@ __all__ = [
     "w4a8_quantize_act", "w4a8_gemm", "w4a8_gemm_i32", "w4a8_gemm_schedule",
     "w4a8_get_status", "w4a8_debug_timeout_probe", "PackedWeights",
     "w8a8_quantize_weights", "w8a8_gemm", "w8a8_gemm_i32", "w8a8_gemm_schedule",
+    "GroupedPackedWeights", "w4a8_quantize_grouped_weights", "w4a8_grouped_gemm",
+    "w4a8_grouped_gemm_i32", "w4a8_grouped_gemm_schedule",
 ]
 
 OK = 0
@@ -34,6 +36,7 @@ ERR_MISALIGNED = -3
 ERR_CUDA = -5
 ERR_TIMEOUT = -6
 ERR_BAD_PACKED = -7
+ERR_BAD_OFFSETS = -8
 
 W4A8_FLAG_PDL = 1  # programmatic dependent launch (see include/w4a8.h)
 
@@ -78,6 +81,9 @@ def lib():
             "w8a8_gemm": ([p, p, p, p, i32, i32, i32, p, _ct.c_uint, p], i32),
             "w8a8_gemm_i32": ([p, p, i32, i32, i32, p, p], i32),
             "w8a8_gemm_schedule": ([i32, i32, i32, p, p, p], i32),
+            "w4a8_grouped_gemm": ([p, p, p, i32, p, i32, i32, i32, i32, p, _ct.c_uint, p], i32),
+            "w4a8_grouped_gemm_i32": ([p, p, i32, p, i32, i32, i32, i32, p, p], i32),
+            "w4a8_grouped_gemm_schedule": ([i32, i32, i32, i32, i32, p, p, p], i32),
             "w4a8_get_status": ([p], i32),
             "w4a8_debug_timeout_probe": ([ll, p], i32),
         }
@@ -218,6 +224,78 @@ def w4a8_gemm_schedule(M, N, K):
     t, s, c = _ct.c_int(0), _ct.c_int(0), _ct.c_int(0)
     _check(lib().w4a8_gemm_schedule(int(M), int(N), int(K), _ct.byref(t), _ct.byref(s),
                                     _ct.byref(c)), "w4a8_gemm_schedule")
+    return t.value, s.value, c.value
+
+
+class GroupedPackedWeights:
+    """Packed LQQ weights of `groups` experts of one shape, back to back in
+    one uint8 CUDA tensor (the layout w4a8_grouped_gemm reads)."""
+
+    def __init__(self, data, groups, N, K, group):
+        self.data, self.groups = data, int(groups)
+        self.N, self.K, self.group = int(N), int(K), int(group)
+        self.expert_bytes = w4a8_packed_weight_bytes(N, K, group)
+
+    def expert(self, g):
+        """The PackedWeights view of expert g (shares memory)."""
+        b = self.expert_bytes
+        return PackedWeights(self.data[g * b:(g + 1) * b], self.N, self.K, self.group)
+
+
+def w4a8_quantize_grouped_weights(W, group=64, stream=None):
+    """Quantize fp32 expert weights W [E, N, K] into one grouped buffer."""
+    if not isinstance(W, _torch.Tensor) or W.dim() != 3:
+        raise TypeError("W must be a 3D [E, N, K] CUDA tensor")
+    E, N, K = W.shape
+    b = w4a8_packed_weight_bytes(N, K, group)
+    if b == 0:
+        raise W4A8Error("w4a8_packed_weight_bytes", ERR_UNSUPPORTED_SHAPE)
+    data = _torch.empty(E * b, dtype=_torch.uint8, device=W.device)
+    for g in range(E):
+        w4a8_quantize_weights(W[g], group=group, out=data[g * b:(g + 1) * b], stream=stream)
+    return GroupedPackedWeights(data, E, N, K, group)
+
+
+def _grouped_args(Xq, gw, offsets, max_rows):
+    _need(Xq, _torch.int8, 2, "Xq")
+    _need(offsets, _torch.int32, 1, "offsets")
+    M, K = Xq.shape
+    if K != gw.K or offsets.numel() != gw.groups + 1:
+        raise ValueError("Xq has K=%d (weights K=%d); offsets needs %d entries"
+                         % (K, gw.K, gw.groups + 1))
+    max_rows = M if max_rows is None else int(max_rows)
+    return M, K, max_rows
+
+
+def w4a8_grouped_gemm(Xq, s_x, gw, offsets, max_rows=None, out=None, stream=None, flags=0):
+    """Grouped (mixture-of-experts) W4A8 GEMM: rows offsets[g]..offsets[g+1]-1
+    of Xq use expert g of ``gw``.  ``offsets`` is an int32 CUDA tensor of
+    groups + 1 entries; ``max_rows`` bounds any group's rows (default M)."""
+    _need(s_x, _torch.float32, 1, "s_x")
+    M, K, max_rows = _grouped_args(Xq, gw, offsets, max_rows)
+    Y = out if out is not None else _torch.empty(M, gw.N, dtype=_torch.bfloat16, device=Xq.device)
+    _check(lib().w4a8_grouped_gemm(_ptr(Xq), _ptr(s_x), _ptr(gw.data), gw.groups, _ptr(offsets),
+                                   M, max_rows, gw.N, K, _ptr(Y), int(flags), _stream(stream)),
+           "w4a8_grouped_gemm")
+    return Y
+
+
+def w4a8_grouped_gemm_i32(Xq, gw, offsets, max_rows=None, out=None, stream=None):
+    """Exact INT32 accumulators of the grouped W4A8 GEMM."""
+    M, K, max_rows = _grouped_args(Xq, gw, offsets, max_rows)
+    acc = out if out is not None else _torch.empty(M, gw.N, dtype=_torch.int32, device=Xq.device)
+    _check(lib().w4a8_grouped_gemm_i32(_ptr(Xq), _ptr(gw.data), gw.groups, _ptr(offsets), M,
+                                       max_rows, gw.N, K, _ptr(acc), _stream(stream)),
+           "w4a8_grouped_gemm_i32")
+    return acc
+
+
+def w4a8_grouped_gemm_schedule(groups, M_total, max_rows, N, K):
+    """(tokens per tile, split-K factor, CTAs launched) of the grouped kernel."""
+    t, s, c = _ct.c_int(0), _ct.c_int(0), _ct.c_int(0)
+    _check(lib().w4a8_grouped_gemm_schedule(int(groups), int(M_total), int(max_rows), int(N),
+                                            int(K), _ct.byref(t), _ct.byref(s), _ct.byref(c)),
+           "w4a8_grouped_gemm_schedule")
     return t.value, s.value, c.value
 
 

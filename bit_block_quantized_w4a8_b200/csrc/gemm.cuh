@@ -67,6 +67,14 @@ struct GemmParams {
   uint32_t x_tx_bytes;    // bytes of one activation box (rows * 128)
   unsigned long long wait_limit_ns;
   const PackedHeader* hdr;  // checked against (N, K) before any store
+  // Grouped GEMM (mixture-of-experts): rows [offsets[g], offsets[g+1]) of
+  // Xq / Y belong to group g, whose packed weights start group_bytes * g
+  // after `hdr`.  M is then the bound on rows per group, m_total the number
+  // of rows of Xq / Y, and m_tiles the number of token-tile slots launched
+  // (each slot takes the next token tile that holds rows, in group order).
+  const int* offsets;     // [groups + 1] on the device, or nullptr (dense)
+  size_t group_bytes;
+  int m_total, groups;
 };
 
 template <int T, int SS, int AS, int DQG, bool PUSH = false, bool W8 = false>
@@ -165,16 +173,64 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
   float* sx_s = reinterpret_cast<float*>(smem + C::kOffSx);
 
   // tile coordinates: the splits of a tile are consecutive blocks (one
-  // cluster), then channel blocks, then token blocks
+  // cluster), then channel blocks, then token blocks (then groups)
   const int split = blockIdx.x % p.splits;
   const int tile = blockIdx.x / p.splits;
   const int n_tile = tile % p.n_tiles;
-  const int m_tile = tile / p.n_tiles;
   const int kt0 = split * p.kt_per_split;
   const int kt1 = min(kt0 + p.kt_per_split, p.kt_total);
   const int nk = kt1 - kt0;
-  const int m0 = m_tile * T;
   const uint64_t lim = p.wait_limit_ns;
+  // rows of this tile: row_base .. row_base + t_valid - 1 of Xq / Y
+  int row_base, t_valid;
+  const uint8_t* w_tiles = p.tiles;
+  const float* w_scale = p.s_w;
+  const PackedHeader* w_hdr = p.hdr;
+  if (p.offsets == nullptr) {
+    row_base = (tile / p.n_tiles) * T;
+    t_valid = min(T, p.M - row_base);
+  } else {
+    // Grouped: the row offsets may be written by the preceding kernel.  Token
+    // tile slot `a` is the a-th tile that holds rows, counting group by
+    // group.  Every CTA checks every group's offsets, so a call with an
+    // invalid group stores nothing.  All CTAs of a cluster (the splits of
+    // one tile) take the same branch, so a slot without work leaves before
+    // any cluster barrier.
+    pdl_wait();
+    int a = tile / p.n_tiles;
+    int g = -1, m_tile = 0, r0 = 0, r1 = 0;
+    bool bad = false;
+    for (int q = 0; q < p.groups; ++q) {
+      const int q0 = p.offsets[q], q1 = p.offsets[q + 1];
+      if (q0 < 0 || q1 < q0 || q1 > p.m_total || q1 - q0 > p.M) {
+        bad = true;
+        break;
+      }
+      const int cnt = (q1 - q0 + T - 1) / T;
+      if (g < 0) {
+        if (a < cnt) {
+          g = q;
+          m_tile = a;
+          r0 = q0;
+          r1 = q1;
+        } else {
+          a -= cnt;
+        }
+      }
+    }
+    if (bad) {
+      if (threadIdx.x == 0) record_status(kDevBadOffsets);
+      return;
+    }
+    if (g < 0) return;
+    row_base = r0 + m_tile * T;
+    t_valid = min(T, r1 - row_base);
+    w_tiles += p.group_bytes * g;
+    w_scale = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(w_scale) +
+                                             p.group_bytes * g);
+    w_hdr = reinterpret_cast<const PackedHeader*>(reinterpret_cast<const uint8_t*>(w_hdr) +
+                                                  p.group_bytes * g);
+  }
 
   // Every warp reaches a CTA-wide barrier converged: an aligned barrier
   // reached by a warp in pieces (one lane late) can complete early and
@@ -227,7 +283,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     }
     const uint64_t pol = l2_policy_evict_first();
     const uint8_t* wsrc = W8 ? nullptr
-                             : p.tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
+                             : w_tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
     // one weight stage: a bulk copy of the packed tile, or a TMA box of
     // 128 channels x 128 k of the INT8 matrix
     auto load_w = [&](int it, int s) {
@@ -251,7 +307,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     pdl_wait();  // activations are produced by the preceding kernel
     if (leader) {
       for (int it = 0; it < pre; ++it)
-        tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
+        tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, row_base,
                     bar_full + 8 * it);
     }
     issued = pre;
@@ -263,7 +319,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
       if (leader) {
         mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         load_w(it, s);
-        tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, m0,
+        tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, row_base,
                     bar_full + 8 * s);
       }
       __syncwarp();
@@ -318,10 +374,10 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     const int n = n_tile * kTileN + r;
     // loads needed only by the epilogue, issued before the main loop so
     // their latency is hidden
-    const float swn = (p.Y && n < p.N) ? __ldg(p.s_w + n) : 0.0f;  // no scales for INT32 output
+    const float swn = (p.Y && n < p.N) ? __ldg(w_scale + n) : 0.0f;  // no scales for INT32 output
     bool hdr_ok = true;
     if (!W8 && warp == 2 && lane == 0)
-      hdr_ok = p.hdr->magic == kMagic && p.hdr->N == p.N && p.hdr->K == p.K;
+      hdr_ok = w_hdr->magic == kMagic && w_hdr->N == p.N && w_hdr->K == p.K;
     for (int it = dg; !W8 && it < nk; it += DQG) {
       const int s = it % SS, a = it % AS;
       // First the A slot's previous contents must be consumed (its MMAs
@@ -361,8 +417,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     const int et = threadIdx.x - 64;  // epilogue thread index
     pdl_wait();  // s_x and the outputs are ordered after the preceding kernel
     if (p.Y) {
-      for (int i = et; i < T; i += nthr)
-        sx_s[i] = (m0 + i < p.M) ? p.s_x[m0 + i] : 0.0f;
+      for (int i = et; i < T; i += nthr) sx_s[i] = i < t_valid ? p.s_x[row_base + i] : 0.0f;
     }
     warp_wait(bar_acc, 0, abort_flag, lim);
     tc_fence_after();
@@ -384,8 +439,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
           if (n < p.N) {
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
-              const int m = m0 + 16 * j + t;
-              if (m < p.M) store_out(p, m, n, (int32_t)v[t], sx_s[16 * j + t], swn);
+              const int tt = 16 * j + t;
+              if (tt < t_valid) store_out(p, row_base + tt, n, (int32_t)v[t], sx_s[tt], swn);
             }
           }
         }
@@ -408,7 +463,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
       // leader's receive buffer and arrive on its barrier; the leader adds
       // its own partial and runs the epilogue
       cluster_wait();
-      const int t_valid = min(T, p.M - m0);
       const uint32_t red = sbase + C::kOffRed;
       if (split != 0) {
         if (*ep_flag) {
@@ -441,7 +495,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
               for (int t = 0; t < 16; ++t) {
                 const int tt = 16 * j + t;
                 if (tt < t_valid)
-                  store_out(p, m0 + tt, n, (int32_t)v[t] + rb[tt * kTileN + r], sx_s[tt], swn);
+                  store_out(p, row_base + tt, n, (int32_t)v[t] + rb[tt * kTileN + r], sx_s[tt],
+                            swn);
               }
             }
           }
@@ -457,7 +512,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     if (warp >= 2 && *ep_flag) {
       const int nthr = 128 * DQG;
       const int et = threadIdx.x - 64;
-      const int t_valid = min(T, p.M - m0);
       const int total = t_valid * kTileN;
       // slices of whole 16-byte groups (4 consecutive channels of a token)
       const int per = ((total + p.splits - 1) / p.splits + 3) & ~3;
@@ -496,19 +550,19 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
           float4 sw4 = make_float4(0.f, 0.f, 0.f, 0.f);
           if (p.Y) {
             if (!W8) {
-              sw4 = __ldg(reinterpret_cast<const float4*>(p.s_w + n2));
+              sw4 = __ldg(reinterpret_cast<const float4*>(w_scale + n2));
             } else {
-              sw4.x = __ldg(p.s_w + n2);
-              if (n2 + 1 < p.N) sw4.y = __ldg(p.s_w + n2 + 1);
-              if (n2 + 2 < p.N) sw4.z = __ldg(p.s_w + n2 + 2);
-              if (n2 + 3 < p.N) sw4.w = __ldg(p.s_w + n2 + 3);
+              sw4.x = __ldg(w_scale + n2);
+              if (n2 + 1 < p.N) sw4.y = __ldg(w_scale + n2 + 1);
+              if (n2 + 2 < p.N) sw4.z = __ldg(w_scale + n2 + 2);
+              if (n2 + 3 < p.N) sw4.w = __ldg(w_scale + n2 + 3);
             }
           }
           const int32_t av[4] = {acc4[b].x, acc4[b].y, acc4[b].z, acc4[b].w};
           const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            if (n2 + i < p.N) store_out(p, m0 + t, n2 + i, av[i], sx_s[t], swv[i]);
+            if (n2 + i < p.N) store_out(p, row_base + t, n2 + i, av[i], sx_s[t], swv[i]);
         }
       }
     }

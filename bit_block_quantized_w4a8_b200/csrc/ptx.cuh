@@ -12,7 +12,7 @@ namespace w4a8 {
 // record the first error they meet here; w4a8_get_status reads and clears.
 __device__ int g_status = 0;
 
-enum : int { kDevOk = 0, kDevTimeout = -6, kDevBadPacked = -7 };
+enum : int { kDevOk = 0, kDevTimeout = -6, kDevBadPacked = -7, kDevBadOffsets = -8 };
 
 __device__ __forceinline__ void record_status(int code) {
   atomicCAS(&g_status, 0, code);

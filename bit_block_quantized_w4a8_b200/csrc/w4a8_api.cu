@@ -166,7 +166,7 @@ int ctas_per_sm(int T, int kt_per, bool w8) {
 // Ties go to more splits.  W4A8_FORCE_SPLITS=<n> and W4A8_FORCE_TILE=<tokens>
 // (not below the tile M needs) in the environment override the choice
 // (tuning only).
-Schedule choose_schedule(int M, int N, int K, int sms, bool w8) {
+Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_tiles = 0) {
   Schedule s;
   s.T = tile_tokens(M);
   static const int forced_tile = [] {  // tuning experiments only
@@ -179,7 +179,8 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8) {
   s.n_tiles = (N + kTileN - 1) / kTileN;
   s.m_tiles = M > 0 ? (M + s.T - 1) / s.T : 0;
   const int kt = K / kTileK;
-  const long tiles = (long)s.n_tiles * s.m_tiles;
+  // tiles that do work (grouped GEMMs launch more, which leave at once)
+  const long tiles = (long)s.n_tiles * (active_m_tiles > 0 ? active_m_tiles : s.m_tiles);
   const double fill = s.T <= 64 ? (s.T == 16 ? 3.5 : 3.7) : s.T == 128 ? 6.0 : 7.4;
   const double t_cta = w8 ? (s.T == 16 ? 0.35 : s.T == 32 ? 0.40 : s.T == 64 ? 0.45 : 0.35)
                          : (s.T > 64 ? 0.29 : s.T == 16 ? 0.27 : s.T == 32 ? 0.28 : 0.32);
@@ -213,7 +214,24 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8) {
       s.kt_per = per;
     }
   }
-  s.ctas = (int)(tiles * s.splits);
+  s.ctas = (int)((long)s.n_tiles * s.m_tiles * s.splits);
+  return s;
+}
+
+// Grouped GEMM: token tiles are per group and the tile width comes from the
+// bound on rows per group.  At most ceil(M_total / T) + groups - 1 token
+// tiles hold rows (one partial tile per group), no more than M_total and no
+// more than groups x ceil(max_rows / T); that many token-tile slots are
+// launched (slots past the actual tiles leave at once) and the cost model
+// counts them.  Schedule::m_tiles is the number of slots.
+Schedule choose_grouped_schedule(int groups, int m_total, int max_rows, int N, int K, int sms) {
+  Schedule s = choose_schedule(max_rows, N, K, sms, false);
+  long slots = (m_total + s.T - 1) / s.T + groups - 1;
+  if (slots > (long)groups * s.m_tiles) slots = (long)groups * s.m_tiles;
+  if (slots > m_total) slots = m_total;
+  s = choose_schedule(max_rows, N, K, sms, false, slots);
+  s.m_tiles = (int)slots;
+  s.ctas = (int)((long)s.n_tiles * s.m_tiles * s.splits);
   return s;
 }
 
@@ -297,6 +315,10 @@ GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K,
   p.m_tiles = s.m_tiles;
   p.wait_limit_ns = kWaitLimitNs;
   p.hdr = nullptr;
+  p.offsets = nullptr;
+  p.group_bytes = 0;
+  p.m_total = M;
+  p.groups = 0;
   // Only rows that exist are fetched when M < T: the MMA still reads T rows,
   // but rows past M only feed accumulator columns that are never stored.
   const int box_rows = M < s.T ? M : s.T;
@@ -304,22 +326,43 @@ GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K,
   return p;
 }
 
+// Grouped (mixture-of-experts) form of a call; groups == 0 for a dense GEMM.
+struct Groups {
+  int groups = 0;
+  const int* offsets = nullptr;
+  int m_total = 0;
+};
+
+// W4A8 GEMM, dense (M rows) or grouped (g.m_total rows in g.groups groups of
+// at most M rows each).
 int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
-                int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
+                int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream,
+                const Groups& g = Groups()) {
   const int rc = check_common(Xq, s_x, packed, M, N, K, Y, acc, flags);
   if (rc != W4A8_OK || M == 0) return rc;
   const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
   const int dev = current_device();
   if (dev < 0) return W4A8_ERR_CUDA;
-  const Schedule s = choose_schedule(M, N, K, num_sms(dev), false);
+  const Schedule s = g.groups > 0 ? choose_grouped_schedule(g.groups, g.m_total, M, N, K,
+                                                            num_sms(dev))
+                                  : choose_schedule(M, N, K, num_sms(dev), false);
   GemmParams p = make_params(s, s_x, M, N, K, Y, acc);
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   p.tiles = base + tiles_offset_bytes(p.n_pad);
   p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
   p.hdr = reinterpret_cast<const PackedHeader*>(base);
+  const int x_rows = g.groups > 0 ? g.m_total : M;  // rows of Xq / Y
+  if (g.groups > 0) {
+    p.offsets = g.offsets;
+    p.group_bytes = (size_t)packed_bytes(N, K);
+    p.m_total = g.m_total;
+    p.groups = g.groups;
+  }
 
   Maps m;
-  if (!make_act_map(&m.x, Xq, M, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
+  // the box holds min(T, M) rows: every valid row of a tile (grouped: M
+  // bounds each group's rows), and exactly the bytes x_tx_bytes expects
+  if (!make_act_map(&m.x, Xq, x_rows, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
   m.w = m.x;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
@@ -413,6 +456,7 @@ const char* w4a8_status_string(int status) {
     case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
     case W4A8_ERR_TIMEOUT: return "W4A8_ERR_TIMEOUT";
     case W4A8_ERR_BAD_PACKED: return "W4A8_ERR_BAD_PACKED";
+    case W4A8_ERR_BAD_OFFSETS: return "W4A8_ERR_BAD_OFFSETS";
     default: return "W4A8_ERR_UNKNOWN";
   }
 }
@@ -501,6 +545,48 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits, int* 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
   const Schedule s = choose_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev), false);
+  if (tile_tokens) *tile_tokens = s.T;
+  if (splits) *splits = s.splits;
+  if (ctas) *ctas = s.ctas;
+  return W4A8_OK;
+}
+
+int w4a8_grouped_gemm(const int8_t* Xq, const float* s_x, const void* packed, int groups,
+                      const int* offsets, int M_total, int max_rows, int N, int K, uint16_t* Y,
+                      unsigned flags, void* stream) {
+  if (groups < 1 || M_total < 0 || max_rows < 0 || max_rows > M_total) return W4A8_ERR_INVALID_ARG;
+  if (M_total == 0) return (flags & ~(unsigned)W4A8_FLAG_PDL) ? W4A8_ERR_INVALID_ARG : W4A8_OK;
+  if (max_rows == 0 || !offsets || !Y) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(offsets, 4)) return W4A8_ERR_MISALIGNED;
+  Groups g;
+  g.groups = groups;
+  g.offsets = offsets;
+  g.m_total = M_total;
+  return gemm_common(Xq, s_x, packed, max_rows, N, K, Y, nullptr, flags, stream, g);
+}
+
+int w4a8_grouped_gemm_i32(const int8_t* Xq, const void* packed, int groups, const int* offsets,
+                          int M_total, int max_rows, int N, int K, int32_t* acc, void* stream) {
+  if (groups < 1 || M_total < 0 || max_rows < 0 || max_rows > M_total) return W4A8_ERR_INVALID_ARG;
+  if (M_total == 0) return W4A8_OK;
+  if (max_rows == 0 || !offsets || !acc) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(offsets, 4)) return W4A8_ERR_MISALIGNED;
+  Groups g;
+  g.groups = groups;
+  g.offsets = offsets;
+  g.m_total = M_total;
+  return gemm_common(Xq, nullptr, packed, max_rows, N, K, nullptr, acc, 0u, stream, g);
+}
+
+int w4a8_grouped_gemm_schedule(int groups, int M_total, int max_rows, int N, int K,
+                               int* tile_tokens, int* splits, int* ctas) {
+  if (groups < 1 || M_total < 1 || max_rows < 1 || max_rows > M_total || N < 1 || K < 1)
+    return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const Schedule s =
+      choose_grouped_schedule(groups, M_total, max_rows, N, K, dev < 0 ? 148 : num_sms(dev));
   if (tile_tokens) *tile_tokens = s.T;
   if (splits) *splits = s.splits;
   if (ctas) *ctas = s.ctas;

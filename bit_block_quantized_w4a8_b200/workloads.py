@@ -168,3 +168,65 @@ def random_matrix(rows: int, cols: int, seed: int, std: float = 1.0,
     elif kind != "normal":
         raise ValueError(kind)
     return X
+
+
+# ------------------------------------------------- mixture-of-experts layers
+# The pages serve Mixtral-8x7B (skeptic concrete_test).  Its expert layers:
+# 8 experts, hidden 4096, expert width 14336, each token routed to 2 experts.
+# The gate and up projections of an expert are one GEMM (N = 2 x 14336).
+# No router weights exist here: each token's two experts are drawn uniformly
+# without replacement by the seeded generator.
+
+@dataclass(frozen=True)
+class MoEWorkload:
+    name: str
+    seed: int
+    experts: int
+    top_k: int
+    layers: Tuple[Layer, ...]
+    tokens: Tuple[int, ...]
+    w_std: float
+    description: str = ""
+
+
+MOE_WORKLOADS: Dict[str, MoEWorkload] = {
+    w.name: w for w in [
+        MoEWorkload("mixtral_like", 6, 8, 2,
+                    (Layer("gate_up", 28672, 4096), Layer("down", 4096, 14336)),
+                    (1, 16, 64, 512), 0.02,
+                    description="8 experts, top-2, tokens in {1,16,64,512}, X~N(0,1), "
+                                "W~N(0,0.02)"),
+    ]
+}
+
+
+def moe_routing(name: str, tokens: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Rows grouped by expert: (offsets int32 [E+1], token index of each row
+    int64 [tokens * top_k]).  Within an expert, rows keep token order."""
+    w = MOE_WORKLOADS[name]
+    g = _gen(w.seed * 1_000_003 + 31 * tokens + 5)
+    choice = torch.stack([torch.randperm(w.experts, generator=g)[:w.top_k]
+                          for _ in range(tokens)])                    # [tokens, top_k]
+    rows_tok, counts = [], []
+    for e in range(w.experts):
+        t = torch.nonzero((choice == e).any(dim=1)).flatten()
+        rows_tok.append(t)
+        counts.append(t.numel())
+    offsets = torch.zeros(w.experts + 1, dtype=torch.int32)
+    offsets[1:] = torch.cumsum(torch.tensor(counts, dtype=torch.int64), 0).to(torch.int32)
+    return offsets, torch.cat(rows_tok)
+
+
+def moe_expert_weights(name: str, layer: Layer, expert: int) -> torch.Tensor:
+    """W_e ~ N(0, std) fp32 [N, K] of one expert."""
+    w = MOE_WORKLOADS[name]
+    idx = [L.name for L in w.layers].index(layer.name)
+    return make_weights(layer.N, layer.K, w.seed * 1_000_003 + 7919 * idx + 613 * expert + 3,
+                        w.w_std)
+
+
+def moe_activations(name: str, layer: Layer, tokens: int) -> torch.Tensor:
+    """X ~ N(0,1) fp32 [tokens, K], one row per token (not yet grouped)."""
+    w = MOE_WORKLOADS[name]
+    idx = [L.name for L in w.layers].index(layer.name)
+    return make_activations(tokens, layer.K, w.seed * 1_000_003 + 7919 * idx + 104_729 * tokens + 4)

@@ -57,7 +57,8 @@ typedef enum {
   W4A8_ERR_MISALIGNED = -3,        /* see the alignment rule above */
   W4A8_ERR_CUDA = -5,              /* a CUDA runtime call failed */
   W4A8_ERR_TIMEOUT = -6,           /* a device-side bounded wait ran out */
-  W4A8_ERR_BAD_PACKED = -7         /* packed buffer header does not match */
+  W4A8_ERR_BAD_PACKED = -7,        /* packed buffer header does not match */
+  W4A8_ERR_BAD_OFFSETS = -8        /* grouped GEMM: invalid row offsets */
 } w4a8_status;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -163,6 +164,45 @@ int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K,
  */
 int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
                        int* ctas);
+
+/*
+ * ---- Grouped GEMM for mixture-of-experts layers ----
+ * The pages serve Mixtral-8x7B (skeptic's concrete test), whose expert
+ * layers are many W4A8 GEMMs of one shape with a variable number of tokens
+ * each.  One launch covers all of them:
+ *   for every group g and row m in [offsets[g], offsets[g+1]):
+ *     Y[m][n] = bf16_rn( float(acc) * (s_x[m] * s_w_g[n]) ),
+ *     acc = sum_k Xq[m][k] * Wdq_g[n][k]
+ * with the rows of Xq / Y grouped by expert (the caller sorts tokens by
+ * expert; a token routed to two experts appears twice).
+ *   packed:  `groups` packed buffers of one (N, K, group), back to back,
+ *            w4a8_packed_weight_bytes(N, K, group) bytes apart (group g's
+ *            buffer starts g times that many bytes after `packed`).
+ *   offsets: int32 [groups + 1] on the DEVICE: offsets[0] = 0, nondecreasing,
+ *            offsets[groups] = M_total.  It may be written by the preceding
+ *            kernel in the stream (with W4A8_FLAG_PDL the kernel waits for it).
+ *   max_rows: host-side bound on the rows of any one group (1..M_total);
+ *            it sizes the launch and the tile width, so a tight bound is
+ *            faster.  Xq [M_total][K], s_x [M_total], Y [M_total][N].
+ * If any group's offsets are out of order, outside [0, M_total] or span
+ * more than max_rows rows, the call stores nothing and w4a8_get_status
+ * reports W4A8_ERR_BAD_OFFSETS.  The launch has one CTA per token tile that
+ * can hold rows (at most ceil(M_total / T) + groups - 1 of them, T the tile
+ * width) times the channel blocks and splits, so empty experts cost nothing.
+ */
+int w4a8_grouped_gemm(const int8_t* Xq, const float* s_x, const void* packed,
+                      int groups, const int* offsets, int M_total, int max_rows,
+                      int N, int K, uint16_t* Y, unsigned flags, void* stream);
+
+/* The grouped product's exact INT32 accumulators acc [M_total][N]. */
+int w4a8_grouped_gemm_i32(const int8_t* Xq, const void* packed, int groups,
+                          const int* offsets, int M_total, int max_rows, int N,
+                          int K, int32_t* acc, void* stream);
+
+/* Schedule of the grouped kernel (as w4a8_gemm_schedule; ctas counts the
+ * CTAs launched, including token-tile slots that find no rows and exit). */
+int w4a8_grouped_gemm_schedule(int groups, int M_total, int max_rows, int N,
+                               int K, int* tile_tokens, int* splits, int* ctas);
 
 /*
  * ---- W8A8 comparison point ----

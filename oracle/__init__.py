@@ -229,6 +229,38 @@ def w4a8_gemm_sampled(Xq, s_x, wq, ms, ns, group=64):
     return acc, Y
 
 
+def w4a8_grouped_gemm(Xq, s_x, wqs, offsets, group=64):
+    """Grouped product of a mixture-of-experts layer (the pages serve
+    Mixtral-8x7B; skeptic concrete_test): rows [offsets[g], offsets[g+1]) of
+    Xq are multiplied with expert g's weights ``wqs[g]`` (dicts as returned
+    by :func:`quantize_weights`).  Returns (acc int32 [M,N], Y bf16 bits)."""
+    Xq = _c(Xq, _np.int8)
+    s_x = _c(s_x, _np.float32)
+    M = Xq.shape[0]
+    N = wqs[0]["codes"].shape[0]
+    acc = _np.zeros((M, N), _np.int32)
+    Y = _np.zeros((M, N), _np.uint16)
+    for g, wq in enumerate(wqs):
+        r0, r1 = int(offsets[g]), int(offsets[g + 1])
+        if r1 > r0:
+            acc[r0:r1], Y[r0:r1] = w4a8_gemm(Xq[r0:r1], s_x[r0:r1], wq, group)
+    return acc, Y
+
+
+def w4a8_grouped_gemm_sampled(Xq, s_x, wqs, offsets, ms, ns, group=64):
+    """Selected outputs of the grouped product, one by one."""
+    ms = _np.asarray(ms, _np.int64)
+    ns = _np.asarray(ns, _np.int64)
+    acc = _np.empty(ms.shape[0], _np.int32)
+    Y = _np.empty(ms.shape[0], _np.uint16)
+    for g, wq in enumerate(wqs):
+        r0, r1 = int(offsets[g]), int(offsets[g + 1])
+        sel = _np.nonzero((ms >= r0) & (ms < r1))[0]
+        if sel.size:
+            acc[sel], Y[sel] = w4a8_gemm_sampled(Xq, s_x, wq, ms[sel], ns[sel], group)
+    return acc, Y
+
+
 def w8a8_quantize_weights(W):
     """The W8A8 comparison point the review page measures the method against
     (pith summary; forward implication 3): 8-bit weights, one symmetric scale

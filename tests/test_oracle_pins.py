@@ -355,3 +355,33 @@ def test_w8a8_error_bound_against_unquantized_product():
     bound = np.abs(X) @ np.broadcast_to(s_w[:, None] / 2.0, W.shape).T \
         + np.broadcast_to(s_x[:, None] / 2.0, X.shape) @ np.abs(What).T
     assert np.all(np.abs(Yf - ref) <= bound * (1 + 1e-9) + np.abs(Yf) * 2.0 ** -8)
+
+
+# --------------------------------------------- grouped (MoE) GEMM (F4)
+
+def test_grouped_oracle_brute_force():
+    """Every output of the grouped oracle equals its definition written out
+    on the dequantized weights: the expert of row m is the g with
+    offsets[g] <= m < offsets[g+1] (found by a plain scan), and
+    y = s_x[m] s_w_g[n] sum_k Xq[m,k] W8_g[n,k].  Empty groups included."""
+    rng = np.random.default_rng(10)
+    E, N, K = 4, 24, 192
+    offsets = np.array([0, 3, 3, 9, 10], np.int64)
+    X = rng.standard_normal((10, K)).astype(np.float32)
+    Xq, s_x = oracle.quantize_act(X)
+    wqs = [oracle.quantize_weights((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
+           for _ in range(E)]
+    acc, Y = oracle.w4a8_grouped_gemm(Xq, s_x, wqs, offsets)
+    for m in range(10):
+        g = 0
+        while not (offsets[g] <= m < offsets[g + 1]):
+            g += 1
+        W8 = oracle.dequant_weights(wqs[g]["codes"], wqs[g]["s_u8"], wqs[g]["a"])
+        for n in range(N):
+            a = int(np.dot(Xq[m].astype(np.int64), W8[n].astype(np.int64)))
+            assert acc[m, n] == a
+            y = float(s_x[m]) * float(wqs[g]["s_w"][n]) * a
+            assert Y[m, n] == oracle.bf16_from_double(y)
+    ms = np.array([0, 2, 3, 8, 9]); ns = np.array([0, 23, 5, 11, 7])
+    a2, y2 = oracle.w4a8_grouped_gemm_sampled(Xq, s_x, wqs, offsets, ms, ns)
+    assert np.array_equal(a2, acc[ms, ns]) and np.array_equal(y2, Y[ms, ns])
