@@ -775,6 +775,68 @@ def run_moe(args):
     return 0
 
 
+def run_ablation(args):
+    """The ablation study: each kernel variant of ``w4a8_gemm_variant``
+    (one design decision changed against a fixed baseline) timed on decode,
+    mid-size and prefill shapes, as graphs of back-to-back calls
+    (programmatic dependent launch) over rotating weight copies larger than
+    twice the L2.  Writes JSON to ``args.ablation``."""
+    import bit_block_quantized_w4a8_b200 as w4
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    shapes = [("decode_sweep_4096", "square", [1, 16, 256]),
+              ("llama70b_like", "up", [1]),
+              ("llama70b_like", "down", [512]),
+              ("prefill", "square8k", [8192])]
+    variants = ["default", "baseline", "naive_dequant", "serial", "one_group",
+                "group_issues_mma"]
+    out = {"peaks": peaks, "variants": variants, "cases": []}
+    for name, lname, Ms in shapes:
+        layer = [L for L in wl.WORKLOADS[name].layers if L.name == lname][0]
+        N, K = layer.N, layer.K
+        torch.cuda.empty_cache()
+        pk = w4.w4a8_quantize_weights(wl.layer_weights(name, layer).to(dev))
+        ncopy = max(1, min(32, -(-2 * l2 // pk.data.numel())))
+        copies = [pk] + [w4.PackedWeights(pk.data.clone(), N, K, GROUP) for _ in range(ncopy - 1)]
+        for M in Ms:
+            X = wl.layer_activations(name, layer, M).to(dev)
+            Xq, sx = w4.w4a8_quantize_act(X)
+            del X
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            n_in = 8 if M < 4096 else 2
+            t = {}
+            for v in variants:
+                def body(v=v):
+                    for i in range(n_in):
+                        w4.w4a8_gemm_variant(v, Xq, sx, copies[i % ncopy], out=Y, stream=stream,
+                                             flags=PDL)
+                with torch.cuda.stream(stream):
+                    body()
+                stream.synchronize()
+                g = _graph(body, stream)
+                with torch.cuda.stream(stream):
+                    g.replay()
+                reps = max(3, min(50, int(2e-3 / max(1e-6, _time_graph(g, 1, stream)))))
+                t[v] = _time_graph(g, reps, stream) / n_in
+                del g
+            status = w4.w4a8_get_status(stream)
+            base = t["baseline"]
+            case = {"workload": name, "layer": lname, "M": M, "N": N, "K": K, "status": status,
+                    "us": {k: x * 1e6 for k, x in t.items()},
+                    "vs_baseline": {k: x / base for k, x in t.items()},
+                    "tops": {k: gemm_ops(M, N, K) / x / 1e12 for k, x in t.items()}}
+            out["cases"].append(case)
+            print("%-18s %-9s M=%-5d " % (name, lname, M) + "  ".join(
+                "%s %.2fus" % (k, x * 1e6) for k, x in t.items()), flush=True)
+        del copies, pk
+    with open(args.ablation, "w") as f:
+        json.dump(out, f, indent=1)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -796,7 +858,11 @@ def main(argv=None):
     ap.add_argument("--moe", default=None, metavar="PATH",
                     help="time the grouped (mixture-of-experts) GEMM on the Mixtral-like "
                          "layers; write a JSON report to PATH")
+    ap.add_argument("--ablation", default=None, metavar="PATH",
+                    help="time the kernel variants of the ablation study; write JSON to PATH")
     args = ap.parse_args(argv)
+    if args.ablation:
+        return run_ablation(args)
     if args.moe:
         return run_moe(args)
     if args.compare:

@@ -26,7 +26,7 @@ __all__ = [
     "w4a8_get_status", "w4a8_debug_timeout_probe", "PackedWeights",
     "w8a8_quantize_weights", "w8a8_gemm", "w8a8_gemm_i32", "w8a8_gemm_schedule",
     "GroupedPackedWeights", "w4a8_quantize_grouped_weights", "w4a8_grouped_gemm",
-    "w4a8_grouped_gemm_i32", "w4a8_grouped_gemm_schedule",
+    "w4a8_grouped_gemm_i32", "w4a8_grouped_gemm_schedule", "w4a8_gemm_variant", "VARIANTS",
 ]
 
 OK = 0
@@ -39,6 +39,10 @@ ERR_BAD_PACKED = -7
 ERR_BAD_OFFSETS = -8
 
 W4A8_FLAG_PDL = 1  # programmatic dependent launch (see include/w4a8.h)
+
+# kernel variants of the ablation study (W4A8_VARIANT_* in include/w4a8.h)
+VARIANTS = {"default": 0, "baseline": 1, "naive_dequant": 2, "serial": 3, "one_group": 4,
+            "group_issues_mma": 5}
 
 
 class W4A8Error(RuntimeError):
@@ -84,6 +88,7 @@ def lib():
             "w4a8_grouped_gemm": ([p, p, p, i32, p, i32, i32, i32, i32, p, _ct.c_uint, p], i32),
             "w4a8_grouped_gemm_i32": ([p, p, i32, p, i32, i32, i32, i32, p, p], i32),
             "w4a8_grouped_gemm_schedule": ([i32, i32, i32, i32, i32, p, p, p], i32),
+            "w4a8_gemm_variant": ([i32, p, p, p, i32, i32, i32, p, p, _ct.c_uint, p], i32),
             "w4a8_get_status": ([p], i32),
             "w4a8_debug_timeout_probe": ([ll, p], i32),
         }
@@ -348,6 +353,30 @@ def w8a8_gemm_schedule(M, N, K):
     _check(lib().w8a8_gemm_schedule(int(M), int(N), int(K), _ct.byref(t), _ct.byref(s),
                                     _ct.byref(c)), "w8a8_gemm_schedule")
     return t.value, s.value, c.value
+
+
+def w4a8_gemm_variant(variant, Xq, s_x, packed, i32=False, out=None, stream=None, flags=0):
+    """The W4A8 product through one of the ablation study's kernel variants
+    (a name of ``VARIANTS`` or its number): bf16 Y, or with ``i32`` the exact
+    INT32 accumulators."""
+    v = VARIANTS[variant] if isinstance(variant, str) else int(variant)
+    _need(Xq, _torch.int8, 2, "Xq")
+    M, K = Xq.shape
+    if K != packed.K:
+        raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
+    N = packed.N
+    if i32:
+        acc = out if out is not None else _torch.empty(M, N, dtype=_torch.int32, device=Xq.device)
+        rc = lib().w4a8_gemm_variant(v, _ptr(Xq), None, _ptr(packed.data), M, N, K, None,
+                                     _ptr(acc), int(flags), _stream(stream))
+        _check(rc, "w4a8_gemm_variant")
+        return acc
+    _need(s_x, _torch.float32, 1, "s_x")
+    Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
+    rc = lib().w4a8_gemm_variant(v, _ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
+                                 None, int(flags), _stream(stream))
+    _check(rc, "w4a8_gemm_variant")
+    return Y
 
 
 def w4a8_get_status(stream=None):

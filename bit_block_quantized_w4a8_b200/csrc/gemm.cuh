@@ -81,6 +81,13 @@ template <int T, int SS, int AS, int DQG, bool PUSH = false, bool W8 = false>
 struct GemmCfg {
   static_assert(T % 16 == 0 && T >= 16 && T <= 256, "MMA N for M=128");
   static_assert(AS <= SS, "the TMEM ring must not be deeper than the smem ring");
+  // A dequantization group at k tile `it` waits for MMA(it - AS) on the A
+  // slot's barrier.  Its own previous wait (tile it - DQG) guarantees
+  // MMA(it - DQG - AS) done, which covers the slot's previous use
+  // (it - 2 AS) only when AS >= DQG or there is one group; otherwise the
+  // barrier can be two phases behind and the parity test passes on a stale
+  // phase.
+  static_assert(W8 || AS >= DQG || DQG == 1, "A slot ring too shallow for the dequant groups");
   static constexpr int kXBytes = T * kTileK;             // activation tile
   // weight stage: one packed LQQ tile, or a 128 x 128 INT8 tile (W8)
   static constexpr int kWBytes = W8 ? kTileN * kTileK : kTileBytes;
@@ -126,6 +133,36 @@ __device__ __forceinline__ void dequant_chunk(uint4 v, uint32_t s, uint32_t a4,
   }
 }
 
+// Ablation of the dequantization (the pages' argument for IMAD + XOR): each
+// code unpacked on its own, code * s + min in signed 32-bit arithmetic,
+// saturated to INT8 and packed back -- the "naive" route that has to guard
+// against overflow.  Same results as dequant_chunk (the quantizer's bound
+// means nothing saturates), many more instructions.
+__device__ __forceinline__ void dequant_chunk_naive(uint4 v, int s, int mn, uint32_t (&out)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int code = (int)((w[j] >> (8 * b + 4 * h)) & 0xFu);
+        const int val = max(-128, min(127, code * s + mn));
+        packed |= ((uint32_t)val & 0xFFu) << (8 * b);
+      }
+      out[2 * j + h] = packed;
+    }
+  }
+}
+
+// Kernel variants for the ablation study (the production kernel is 0).
+enum : int {
+  kVarDefault = 0,
+  kVarNaiveDequant = 1,  // dequant_chunk_naive instead of IMAD + XOR
+  kVarGroupIssuesMma = 2,  // the dequantization warpgroup issues the MMAs itself
+};
+
 // One output: bf16(acc * (s_x * s_w)) in fp32 with a single rounding, or
 // the exact INT32 accumulator.
 __device__ __forceinline__ void store_out(const GemmParams& p, int m, int n, int32_t a,
@@ -147,12 +184,14 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8>
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8, int V>
 __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, MINB)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_w,  // W8 only
                      const GemmParams p) {
   using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
+  static_assert(V != kVarGroupIssuesMma || (DQG == 1 && !W8),
+                "the issuing warpgroup must see every k tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -331,7 +370,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
         mbar_wait(bar_full + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
     }
     __syncwarp();  // reconverge before any CTA- or cluster-wide barrier
-  } else if (warp == 1) {
+  } else if (warp == 1 && V != kVarGroupIssuesMma) {
     // ---------------------------------------------------------- MMA issuer
     // Whole warp waits, one elected lane issues the MMAs and commits.
     const bool leader = elect_one();
@@ -365,7 +404,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     }
     if (leader) tc_commit(bar_acc);  // also on abort: tracks every MMA issued
     __syncwarp();
-  } else {
+  } else if (warp >= 2) {
     // --------------------------------------------- dequantization warps
     const int dg = (warp - 2) / 4;         // dequant group
     const int quarter = warp & 3;          // TMEM lane quarter of this warp
@@ -402,14 +441,40 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
       for (int c = 0; c < 4; ++c) {
         const uint32_t sh = (c < 2) ? 0 : 16;
         const uint32_t sc = (prm >> sh) & 0xFFu;
-        const uint32_t a4 = ((prm >> (sh + 8)) & 0xFFu) * 0x01010101u;
-        dequant_chunk(v[c], sc, a4, *reinterpret_cast<uint32_t(*)[8]>(out + 8 * c));
+        if (V == kVarNaiveDequant) {
+          const int mn = (int)((prm >> (sh + 8)) & 0xFFu) - 128;
+          dequant_chunk_naive(v[c], (int)sc, mn, *reinterpret_cast<uint32_t(*)[8]>(out + 8 * c));
+        } else {
+          const uint32_t a4 = ((prm >> (sh + 8)) & 0xFFu) * 0x01010101u;
+          dequant_chunk(v[c], sc, a4, *reinterpret_cast<uint32_t(*)[8]>(out + 8 * c));
+        }
       }
       tmem_st_x32(lane_base + C::kA0 + 32 * a, out);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_dq + 8 * a);
+      if (V == kVarGroupIssuesMma && warp == 2) {
+        // ablation: the first warp of the (single) dequantization group
+        // issues this k tile's MMAs once all four quarters are in TMEM
+        if (!warp_wait(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
+          const uint32_t a_tmem = tmem + C::kA0 + 32 * a;
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 32; ++kk)
+            mma_i8_ts(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc_i8(128, T),
+                      (it | kk) != 0);
+          tc_commit(bar_empty + 8 * s);
+          tc_commit(bar_afree + 8 * a);
+        }
+        __syncwarp();
+      }
+    }
+    if (V == kVarGroupIssuesMma && warp == 2) {
+      if (elect_one()) tc_commit(bar_acc);  // also on abort: tracks every MMA issued
+      __syncwarp();
     }
 
     // -------------------------------------------------------- epilogue

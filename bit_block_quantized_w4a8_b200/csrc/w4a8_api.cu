@@ -99,13 +99,14 @@ bool make_w8_map(CUtensorMap* map, const int8_t* Wq, int N, int K) {
 }
 
 // -------------------------------------------------- kernel attributes
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false>
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
+          int V = kVarDefault>
 cudaError_t ensure_smem_attr() {
   using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
-    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8>,
+    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -166,9 +167,10 @@ int ctas_per_sm(int T, int kt_per, bool w8) {
 // Ties go to more splits.  W4A8_FORCE_SPLITS=<n> and W4A8_FORCE_TILE=<tokens>
 // (not below the tile M needs) in the environment override the choice
 // (tuning only).
-Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_tiles = 0) {
+Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_tiles = 0,
+                         int force_T = 0) {
   Schedule s;
-  s.T = tile_tokens(M);
+  s.T = force_T > 0 ? force_T : tile_tokens(M);
   static const int forced_tile = [] {  // tuning experiments only
     const char* e = getenv("W4A8_FORCE_TILE");
     return e ? atoi(e) : 0;
@@ -270,12 +272,13 @@ struct Maps {
   CUtensorMap x, w;
 };
 
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false>
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
+          int V = kVarDefault>
 cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream_t st,
                         bool pdl) {
   using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
-  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8>;
-  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8>();
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V>;
+  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8, V>();
   if (ea != cudaSuccess) return ea;
   return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, p.splits, m.x,
                   m.w, p);
@@ -425,6 +428,62 @@ int gemm_w8_common(const int8_t* Xq, const float* s_x, const int8_t* Wq, const f
     case 64: e = launch_gemm<64, 4, 1, 1, 2, false, true>(m, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 3, 1, 1, 2, false, true>(m, p, s.ctas, st, pdl); break;
     default: e = launch_gemm<256, 4, 1, 1, 1, false, true>(m, p, s.ctas, st, pdl); break;
+  }
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+// Ablation study: the same product through kernel variants that each change
+// one design decision against a fixed baseline configuration (16-token tile
+// with the deep ring for M <= 16, else the 256-token tile; gather split-K
+// reduction; the library's schedule).
+int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* packed, int M,
+                 int N, int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
+  if (variant < W4A8_VARIANT_DEFAULT || variant > W4A8_VARIANT_GROUP_ISSUES_MMA)
+    return W4A8_ERR_INVALID_ARG;
+  if (variant == W4A8_VARIANT_DEFAULT)
+    return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream);
+  const int rc = check_common(Xq, s_x, packed, M, N, K, Y, acc, flags);
+  if (rc != W4A8_OK || M == 0) return rc;
+  const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
+  const int dev = current_device();
+  if (dev < 0) return W4A8_ERR_CUDA;
+  const int T = M <= 16 ? 16 : 256;
+  const Schedule s = choose_schedule(M, N, K, num_sms(dev), false, 0, T);
+  GemmParams p = make_params(s, s_x, M, N, K, Y, acc);
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  p.tiles = base + tiles_offset_bytes(p.n_pad);
+  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
+  p.hdr = reinterpret_cast<const PackedHeader*>(base);
+  Maps m;
+  if (!make_act_map(&m.x, Xq, M, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
+  m.w = m.x;
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+  // (tokens, smem stages, TMEM A slots, dequant groups, CTAs per SM, push, W8, variant)
+  if (T == 16) {
+    switch (variant) {
+      case W4A8_VARIANT_BASELINE: e = launch_gemm<16, 10, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
+      case W4A8_VARIANT_NAIVE_DEQUANT:
+        e = launch_gemm<16, 10, 4, 2, 2, false, false, kVarNaiveDequant>(m, p, s.ctas, st, pdl);
+        break;
+      case W4A8_VARIANT_SERIAL: e = launch_gemm<16, 10, 1, 1, 2>(m, p, s.ctas, st, pdl); break;
+      case W4A8_VARIANT_ONE_GROUP: e = launch_gemm<16, 10, 4, 1, 2>(m, p, s.ctas, st, pdl); break;
+      default:
+        e = launch_gemm<16, 10, 4, 1, 2, false, false, kVarGroupIssuesMma>(m, p, s.ctas, st, pdl);
+        break;
+    }
+  } else {
+    switch (variant) {
+      case W4A8_VARIANT_BASELINE: e = launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl); break;
+      case W4A8_VARIANT_NAIVE_DEQUANT:
+        e = launch_gemm<256, 5, 4, 2, 1, false, false, kVarNaiveDequant>(m, p, s.ctas, st, pdl);
+        break;
+      case W4A8_VARIANT_SERIAL: e = launch_gemm<256, 5, 1, 1, 1>(m, p, s.ctas, st, pdl); break;
+      case W4A8_VARIANT_ONE_GROUP: e = launch_gemm<256, 5, 4, 1, 1>(m, p, s.ctas, st, pdl); break;
+      default:
+        e = launch_gemm<256, 5, 4, 1, 1, false, false, kVarGroupIssuesMma>(m, p, s.ctas, st, pdl);
+        break;
+    }
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
@@ -591,6 +650,12 @@ int w4a8_grouped_gemm_schedule(int groups, int M_total, int max_rows, int N, int
   if (splits) *splits = s.splits;
   if (ctas) *ctas = s.ctas;
   return W4A8_OK;
+}
+
+int w4a8_gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* packed, int M,
+                      int N, int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
+  if (Y && acc) return W4A8_ERR_INVALID_ARG;
+  return gemm_variant(variant, Xq, s_x, packed, M, N, K, Y, acc, flags, stream);
 }
 
 int w8a8_quantize_weights(const float* W, int N, int K, int8_t* Wq, float* s_w, void* stream) {

@@ -166,6 +166,40 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
                        int* ctas);
 
 /*
+ * ---- Ablation variants ----
+ * The review page reports an ablation of the method's parts (referee
+ * significance: LQQ, ImFP and their effect on throughput).  These variants
+ * each change one design decision of this library's kernel against a fixed
+ * baseline, and compute exactly the same result:
+ *   BASELINE          16-token tile with the deep ring (10 stages) for
+ *                     M <= 16, else the 256-token tile; two dequantization
+ *                     warpgroups, a dedicated MMA warp, 4 TMEM weight
+ *                     slots, gather split-K reduction, the library's splits
+ *   NAIVE_DEQUANT     each 4-bit code unpacked on its own, code * s + min in
+ *                     signed 32-bit arithmetic, saturated to INT8 and packed
+ *                     (instead of two instructions per four weights)
+ *   ONE_GROUP         one dequantization warpgroup instead of two
+ *   SERIAL            one dequantization warpgroup and one TMEM weight slot:
+ *                     dequantizing a k tile waits for the MMAs of the
+ *                     previous one (no overlap of the two)
+ *   GROUP_ISSUES_MMA  one dequantization warpgroup that also issues the MMAs
+ *                     (no dedicated MMA warp)
+ * DEFAULT is the library's own choice (w4a8_gemm_ex / w4a8_gemm_i32).
+ * Exactly one of Y (bf16, with s_x) or acc (INT32) is non-NULL.  Other
+ * arguments as for w4a8_gemm_ex.
+ */
+#define W4A8_VARIANT_DEFAULT 0
+#define W4A8_VARIANT_BASELINE 1
+#define W4A8_VARIANT_NAIVE_DEQUANT 2
+#define W4A8_VARIANT_SERIAL 3
+#define W4A8_VARIANT_ONE_GROUP 4
+#define W4A8_VARIANT_GROUP_ISSUES_MMA 5
+
+int w4a8_gemm_variant(int variant, const int8_t* Xq, const float* s_x,
+                      const void* packed, int M, int N, int K, uint16_t* Y,
+                      int32_t* acc, unsigned flags, void* stream);
+
+/*
  * ---- Grouped GEMM for mixture-of-experts layers ----
  * The pages serve Mixtral-8x7B (skeptic's concrete test), whose expert
  * layers are many W4A8 GEMMs of one shape with a variable number of tokens
