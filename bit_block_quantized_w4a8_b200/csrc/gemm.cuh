@@ -75,6 +75,13 @@ struct GemmParams {
   const int* offsets;     // [groups + 1] on the device, or nullptr (dense)
   size_t group_bytes;
   int m_total, groups;
+  // Dense raster: tiles run through bands of `m_band` token tiles, channel
+  // block by channel block, so that a wave of CTAs reuses both operands in
+  // L2 (1 = channel blocks first).
+  int m_band;
+  // Weight tiles are read by one token tile only (stream them through L2
+  // with evict-first), or reused by several (normal priority).
+  int w_stream;
 };
 
 template <int T, int SS, int AS, int DQG, bool PUSH = false, bool W8 = false>
@@ -215,7 +222,18 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
   // cluster), then channel blocks, then token blocks (then groups)
   const int split = blockIdx.x % p.splits;
   const int tile = blockIdx.x / p.splits;
-  const int n_tile = tile % p.n_tiles;
+  int n_tile, m_slot;  // channel block; token tile (grouped: token-tile slot)
+  if (p.offsets == nullptr && p.m_band > 1) {
+    const int span = p.m_band * p.n_tiles;
+    const int m_first = (tile / span) * p.m_band;
+    const int rows = min(p.m_band, p.m_tiles - m_first);
+    const int within = tile % span;
+    n_tile = within / rows;
+    m_slot = m_first + within % rows;
+  } else {
+    n_tile = tile % p.n_tiles;
+    m_slot = tile / p.n_tiles;
+  }
   const int kt0 = split * p.kt_per_split;
   const int kt1 = min(kt0 + p.kt_per_split, p.kt_total);
   const int nk = kt1 - kt0;
@@ -226,7 +244,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
   const float* w_scale = p.s_w;
   const PackedHeader* w_hdr = p.hdr;
   if (p.offsets == nullptr) {
-    row_base = (tile / p.n_tiles) * T;
+    row_base = m_slot * T;
     t_valid = min(T, p.M - row_base);
   } else {
     // Grouped: the row offsets may be written by the preceding kernel.  Token
@@ -236,7 +254,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     // one tile) take the same branch, so a slot without work leaves before
     // any cluster barrier.
     pdl_wait();
-    int a = tile / p.n_tiles;
+    int a = m_slot;
     int g = -1, m_tile = 0, r0 = 0, r1 = 0;
     bool bad = false;
     for (int q = 0; q < p.groups; ++q) {
@@ -320,7 +338,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
       prefetch_tensormap(&tmap_x);
       if (W8) prefetch_tensormap(&tmap_w);
     }
-    const uint64_t pol = l2_policy_evict_first();
+    const uint64_t pol = p.w_stream ? l2_policy_evict_first() : l2_policy_evict_normal();
     const uint8_t* wsrc = W8 ? nullptr
                              : w_tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
     // one weight stage: a bulk copy of the packed tile, or a TMA box of

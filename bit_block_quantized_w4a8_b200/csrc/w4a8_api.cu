@@ -121,6 +121,7 @@ struct Schedule {
 };
 
 constexpr int kMaxSplits = 8;  // portable thread-block cluster size
+constexpr int kRasterBand = 8;  // token tiles per raster band (dense GEMMs)
 
 // Tokens per tile: the smallest MMA N (multiple of 16, up to 256) that
 // covers M, so decode shapes do no wasted MMA work beyond 16 tokens.
@@ -165,8 +166,7 @@ int ctas_per_sm(int T, int kt_per, bool w8) {
 // - the cluster reduction costs ~0.1 us per halving step plus, for the
 //   gather form, the partial tile (0.005 us per token column).
 // Ties go to more splits.  W4A8_FORCE_SPLITS=<n> and W4A8_FORCE_TILE=<tokens>
-// (not below the tile M needs) in the environment override the choice
-// (tuning only).
+// in the environment override the choice (tuning only).
 Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_tiles = 0,
                          int force_T = 0) {
   Schedule s;
@@ -175,9 +175,9 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_ti
     const char* e = getenv("W4A8_FORCE_TILE");
     return e ? atoi(e) : 0;
   }();
-  if (forced_tile == 16 || forced_tile == 32 || forced_tile == 64 || forced_tile == 128 ||
-      forced_tile == 256)
-    if (forced_tile >= s.T) s.T = forced_tile;
+  if (force_T == 0 && (forced_tile == 16 || forced_tile == 32 || forced_tile == 64 ||
+                       forced_tile == 128 || forced_tile == 256))
+    s.T = forced_tile;
   s.n_tiles = (N + kTileN - 1) / kTileN;
   s.m_tiles = M > 0 ? (M + s.T - 1) / s.T : 0;
   const int kt = K / kTileK;
@@ -322,6 +322,12 @@ GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K,
   p.group_bytes = 0;
   p.m_total = M;
   p.groups = 0;
+  // Bands of up to 8 token tiles: a wave of 148 CTAs then spans about 18
+  // channel blocks x 8 token tiles, whose weights and activations stay in
+  // L2 while the wave reuses them.  Weights read by one token tile only are
+  // streamed with an evict-first hint.
+  p.m_band = s.m_tiles < kRasterBand ? s.m_tiles : kRasterBand;
+  p.w_stream = s.m_tiles == 1 ? 1 : 0;
   // Only rows that exist are fetched when M < T: the MMA still reads T rows,
   // but rows past M only feed accumulator columns that are never stored.
   const int box_rows = M < s.T ? M : s.T;
@@ -360,6 +366,8 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     p.group_bytes = (size_t)packed_bytes(N, K);
     p.m_total = g.m_total;
     p.groups = g.groups;
+    p.m_band = 1;
+    p.w_stream = M <= s.T ? 1 : 0;  // one token tile per group
   }
 
   Maps m;
