@@ -792,7 +792,7 @@ def run_ablation(args):
               ("llama70b_like", "down", [512]),
               ("prefill", "square8k", [8192])]
     variants = ["default", "baseline", "naive_dequant", "serial", "one_group",
-                "group_issues_mma"]
+                "group_issues_mma", "cta_pair"]
     out = {"peaks": peaks, "variants": variants, "cases": []}
     for name, lname, Ms in shapes:
         layer = [L for L in wl.WORKLOADS[name].layers if L.name == lname][0]
@@ -809,6 +809,8 @@ def run_ablation(args):
             n_in = 8 if M < 4096 else 2
             t = {}
             for v in variants:
+                if v == "cta_pair" and (M < 256 or (-(-N // 128)) % 2):
+                    continue  # the pair form needs full 256-token tiles, paired channel blocks
                 def body(v=v):
                     for i in range(n_in):
                         w4.w4a8_gemm_variant(v, Xq, sx, copies[i % ncopy], out=Y, stream=stream,

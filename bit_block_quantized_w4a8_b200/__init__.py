@@ -42,7 +42,7 @@ W4A8_FLAG_PDL = 1  # programmatic dependent launch (see include/w4a8.h)
 
 # kernel variants of the ablation study (W4A8_VARIANT_* in include/w4a8.h)
 VARIANTS = {"default": 0, "baseline": 1, "naive_dequant": 2, "serial": 3, "one_group": 4,
-            "group_issues_mma": 5}
+            "group_issues_mma": 5, "cta_pair": 6}
 
 
 class W4A8Error(RuntimeError):

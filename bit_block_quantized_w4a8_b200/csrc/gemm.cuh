@@ -84,9 +84,14 @@ struct GemmParams {
   int w_stream;
 };
 
-template <int T, int SS, int AS, int DQG, bool PUSH = false, bool W8 = false>
+template <int T, int SS, int AS, int DQG, bool PUSH = false, bool W8 = false,
+          bool PAIR = false>
 struct GemmCfg {
   static_assert(T % 16 == 0 && T >= 16 && T <= 256, "MMA N for M=128");
+  // PAIR: a 2-CTA cluster computes 256 channels x T tokens with CTA-pair
+  // MMAs; each CTA holds its 128 channels (A and D in its tensor memory) and
+  // loads half of the T tokens (B).
+  static_assert(!PAIR || (T == 256 && !W8 && !PUSH), "CTA pairs use the 256-token tile");
   static_assert(AS <= SS, "the TMEM ring must not be deeper than the smem ring");
   // A dequantization group at k tile `it` waits for MMA(it - AS) on the A
   // slot's barrier.  Its own previous wait (tile it - DQG) guarantees
@@ -95,13 +100,14 @@ struct GemmCfg {
   // barrier can be two phases behind and the parity test passes on a stale
   // phase.
   static_assert(W8 || AS >= DQG || DQG == 1, "A slot ring too shallow for the dequant groups");
-  static constexpr int kXBytes = T * kTileK;             // activation tile
+  static constexpr int kXBytes = (PAIR ? T / 2 : T) * kTileK;  // activation tile
   // weight stage: one packed LQQ tile, or a 128 x 128 INT8 tile (W8)
   static constexpr int kWBytes = W8 ? kTileN * kTileK : kTileBytes;
   static constexpr int kThreads = (2 + 4 * DQG) * 32;
   static constexpr int kA0 = T < 32 ? 32 : T;             // first A column
   static constexpr int kColsUsed = W8 ? kA0 : kA0 + 32 * AS;
-  static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
+  // a pair allocates all 512 columns, so both CTAs get column address 0
+  static constexpr int kTmemCols = PAIR ? 512 : kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
                                    : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
   static_assert(kColsUsed <= 512, "TMEM columns");
   // shared memory: x tiles | w tiles | barriers | misc | s_x cache
@@ -191,12 +197,12 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8, int V>
-__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, MINB)
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8, int V, bool PAIR>
+__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThreads, MINB)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_w,  // W8 only
                      const GemmParams p) {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
   static_assert(V != kVarGroupIssuesMma || (DQG == 1 && !W8),
                 "the issuing warpgroup must see every k tile");
   extern __shared__ uint8_t smem_raw[];
@@ -220,20 +226,25 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
 
   // tile coordinates: the splits of a tile are consecutive blocks (one
   // cluster), then channel blocks, then token blocks (then groups)
-  const int split = blockIdx.x % p.splits;
-  const int tile = blockIdx.x / p.splits;
+  // A CTA pair (PAIR; no split-K) is two consecutive blocks covering
+  // channel blocks 2j and 2j + 1 of the same token tile.
+  const int rank = PAIR ? (int)cluster_ctarank() : 0;
+  const int split = PAIR ? 0 : blockIdx.x % p.splits;
+  const int tile = PAIR ? blockIdx.x >> 1 : blockIdx.x / p.splits;
+  const int n_units = PAIR ? p.n_tiles >> 1 : p.n_tiles;  // channel blocks (pairs) per row
   int n_tile, m_slot;  // channel block; token tile (grouped: token-tile slot)
   if (p.offsets == nullptr && p.m_band > 1) {
-    const int span = p.m_band * p.n_tiles;
+    const int span = p.m_band * n_units;
     const int m_first = (tile / span) * p.m_band;
     const int rows = min(p.m_band, p.m_tiles - m_first);
     const int within = tile % span;
     n_tile = within / rows;
     m_slot = m_first + within % rows;
   } else {
-    n_tile = tile % p.n_tiles;
-    m_slot = tile / p.n_tiles;
+    n_tile = tile % n_units;
+    m_slot = tile / n_units;
   }
+  if (PAIR) n_tile = 2 * n_tile + rank;
   const int kt0 = split * p.kt_per_split;
   const int kt1 = min(kt0 + p.kt_per_split, p.kt_total);
   const int nk = kt1 - kt0;
@@ -299,7 +310,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
         mbar_init(bar_empty + 8 * s, 1);
       }
       for (int a = 0; a < AS; ++a) {
-        mbar_init(bar_dq + 8 * a, 4);
+        // the even CTA of a pair also counts the odd CTA's relayed arrival
+        mbar_init(bar_dq + 8 * a, PAIR && rank == 0 ? 8 : 4);
         mbar_init(bar_afree + 8 * a, 1);
       }
       mbar_init(bar_acc, 1);
@@ -311,8 +323,13 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     }
     __syncwarp();
   } else if (warp == 1) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (push && split == 0) {  // the leader's receive buffer starts at zero
     int4* red = reinterpret_cast<int4*>(smem + C::kOffRed);
@@ -326,6 +343,19 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
   // every CTA of the cluster announces that its barriers and buffers are
   // initialised; the matching wait comes just before the first remote access
   if (push) cluster_arrive();
+  if (PAIR) {
+    // both CTAs' barriers exist before any cross-CTA arrival, and both
+    // tensor-memory allocations start at the same column (the pair MMA
+    // addresses both with one address); otherwise the pair does no work
+    cluster_sync_all();
+    const uint32_t other = (uint32_t)dsmem_ld_s32(
+        dsmem_map(smem_u32(const_cast<uint32_t*>(tmem_slot)), (uint32_t)(rank ^ 1)));
+    if (other != tmem && threadIdx.x == 0) {
+      record_status(kDevTimeout);
+      *abort_flag = 1;
+    }
+    __syncthreads();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -364,8 +394,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     pdl_wait();  // activations are produced by the preceding kernel
     if (leader) {
       for (int it = 0; it < pre; ++it)
-        tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, row_base,
-                    bar_full + 8 * it);
+        tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
+                    row_base + rank * (T / 2), bar_full + 8 * it);
     }
     issued = pre;
     __syncwarp();
@@ -376,8 +406,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
       if (leader) {
         mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         load_w(it, s);
-        tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK, row_base,
-                    bar_full + 8 * s);
+        tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
+                    row_base + rank * (T / 2), bar_full + 8 * s);
       }
       __syncwarp();
       issued = it + 1;
@@ -388,6 +418,39 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
         mbar_wait(bar_full + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
     }
     __syncwarp();  // reconverge before any CTA- or cluster-wide barrier
+  } else if (warp == 1 && PAIR) {
+    // ------------------------------------------- MMA issuer of a CTA pair
+    // The even CTA issues every MMA for both: it waits for both CTAs'
+    // weight slots (its dq barrier counts one arrival relayed from the odd
+    // CTA, which also means that CTA's token half of the stage has landed)
+    // and for its own stage; the completions arrive on the barriers of both
+    // CTAs.  In the odd CTA this warp is the relay: once its four
+    // dequantization warps have arrived locally on a slot it makes the one
+    // cluster-scope release arrive on the even CTA's barrier, keeping that
+    // fence off the dequantization warps.
+    if (rank == 0) {
+      const bool leader = elect_one();
+      constexpr uint32_t idesc = idesc_i8(256, T);
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % SS, a = it % AS;
+        if (!warp_wait<true>(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
+        if (!warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
+          const uint32_t a_tmem = tmem + C::kA0 + 32 * a;
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 32; ++kk)
+            mma_i8_ts_pair(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc,
+                           (it | kk) != 0);
+          tc_commit_pair(bar_empty + 8 * s);
+          tc_commit_pair(bar_afree + 8 * a);
+        }
+        __syncwarp();
+      }
+      if (leader) tc_commit_pair(bar_acc);  // also on abort: tracks every MMA issued
+      __syncwarp();
+    }
   } else if (warp == 1 && V != kVarGroupIssuesMma) {
     // ---------------------------------------------------------- MMA issuer
     // Whole warp waits, one elected lane issues the MMAs and commits.
@@ -471,7 +534,12 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dq + 8 * a);
+      if (lane == 0) {
+        if (PAIR && rank != 0)
+          mbar_arrive_remote_relaxed(dsmem_map(bar_dq + 8 * a, 0));
+        else
+          mbar_arrive(bar_dq + 8 * a);
+      }
       if (V == kVarGroupIssuesMma && warp == 2) {
         // ablation: the first warp of the (single) dequantization group
         // issues this k tile's MMAs once all four quarters are in TMEM
@@ -666,10 +734,16 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8>::kThreads, M
     warp_wait(bar_done, 0, nullptr, lim);
     if (*abort_flag) warp_wait(bar_acc, 0, nullptr, lim);
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, C::kTmemCols);
+    else
+      tmem_dealloc(tmem, C::kTmemCols);
   }
   __syncwarp();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still arrive on its
+  // barriers
+  if (PAIR) cluster_sync_all();
 }
 
 }  // namespace w4a8

@@ -100,13 +100,13 @@ bool make_w8_map(CUtensorMap* map, const int8_t* Wq, int N, int K) {
 
 // -------------------------------------------------- kernel attributes
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
-          int V = kVarDefault>
+          int V = kVarDefault, bool PAIR = false>
 cudaError_t ensure_smem_attr() {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
-    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V>,
+    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -168,7 +168,7 @@ int ctas_per_sm(int T, int kt_per, bool w8) {
 // Ties go to more splits.  W4A8_FORCE_SPLITS=<n> and W4A8_FORCE_TILE=<tokens>
 // in the environment override the choice (tuning only).
 Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_tiles = 0,
-                         int force_T = 0) {
+                         int force_T = 0, int force_splits = 0) {
   Schedule s;
   s.T = force_T > 0 ? force_T : tile_tokens(M);
   static const int forced_tile = [] {  // tuning experiments only
@@ -209,7 +209,8 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_ti
     const double tok = M < s.T ? M : s.T;
     const double red = lg * (0.1 + (push ? 0.05 : 0.005 * tok));
     double cost = waves * (fill + per * t_tile) + red;
-    if (forced > 0) cost = (eff == forced) ? 0.0 : 1e6 + cost;
+    const int want = force_splits > 0 ? force_splits : forced;
+    if (want > 0) cost = (eff == want) ? 0.0 : 1e6 + cost;
     if (cost <= best) {
       best = cost;
       s.splits = eff;
@@ -273,15 +274,37 @@ struct Maps {
 };
 
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
-          int V = kVarDefault>
+          int V = kVarDefault, bool PAIR = false>
 cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream_t st,
                         bool pdl) {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8>;
-  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V>;
-  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8, V>();
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR>;
+  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR>();
   if (ea != cudaSuccess) return ea;
-  return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl, p.splits, m.x,
-                  m.w, p);
+  return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl,
+                  PAIR ? 2 : p.splits, m.x, m.w, p);
+}
+
+// The CTA-pair form of the 256-token tile (two CTAs share each token tile:
+// each holds 128 channels and loads half of the tokens, so a stage is
+// 16 KB of activations instead of 32 KB and the ring is 8 deep instead of
+// 5): taken for dense calls without split-K whose channel blocks pair up
+// and whose token tiles are full height.  W4A8_PAIR=0 in the environment
+// turns it off (tuning only).
+bool use_pair(const Schedule& s, int M) {
+  static const bool enabled = [] {
+    const char* v = getenv("W4A8_PAIR");
+    return !(v && v[0] == '0');
+  }();
+  return enabled && s.T == 256 && s.splits == 1 && s.n_tiles % 2 == 0 && M >= 256;
+}
+
+// Pair launch: the activation box is the CTA's half of the token tile.
+cudaError_t launch_pair(const int8_t* Xq, int M, int K, Maps& m, GemmParams& p, int ctas,
+                        cudaStream_t st, bool pdl) {
+  if (!make_act_map(&m.x, Xq, M, K, 128)) return cudaErrorInvalidValue;
+  p.x_tx_bytes = 128u * kTileK;
+  return launch_gemm<256, 8, 4, 2, 1, false, false, kVarDefault, true>(m, p, ctas, st, pdl);
 }
 
 // Checks shared by both weight formats; fills the launch-independent part
@@ -397,7 +420,11 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     case 32: e = launch_gemm<32, 8, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
     case 64: e = launch_gemm<64, 6, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 4, 4, 2, 2>(m, p, s.ctas, st, pdl); break;  // tuning only
-    default: e = launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl); break;
+    default:
+      e = (g.groups == 0 && use_pair(s, M))
+              ? launch_pair(Xq, M, K, m, p, s.ctas, st, pdl)
+              : launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl);
+      break;
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
@@ -446,7 +473,7 @@ int gemm_w8_common(const int8_t* Xq, const float* s_x, const int8_t* Wq, const f
 // reduction; the library's schedule).
 int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* packed, int M,
                  int N, int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
-  if (variant < W4A8_VARIANT_DEFAULT || variant > W4A8_VARIANT_GROUP_ISSUES_MMA)
+  if (variant < W4A8_VARIANT_DEFAULT || variant > W4A8_VARIANT_CTA_PAIR)
     return W4A8_ERR_INVALID_ARG;
   if (variant == W4A8_VARIANT_DEFAULT)
     return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream);
@@ -456,7 +483,10 @@ int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* pa
   const int dev = current_device();
   if (dev < 0) return W4A8_ERR_CUDA;
   const int T = M <= 16 ? 16 : 256;
-  const Schedule s = choose_schedule(M, N, K, num_sms(dev), false, 0, T);
+  const bool pair = variant == W4A8_VARIANT_CTA_PAIR;
+  if (pair && (T != 256 || ((N + kTileN - 1) / kTileN) % 2 != 0 || M < 256))
+    return W4A8_ERR_UNSUPPORTED_SHAPE;
+  const Schedule s = choose_schedule(M, N, K, num_sms(dev), false, 0, T, pair ? 1 : 0);
   GemmParams p = make_params(s, s_x, M, N, K, Y, acc);
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   p.tiles = base + tiles_offset_bytes(p.n_pad);
@@ -480,6 +510,8 @@ int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* pa
         e = launch_gemm<16, 10, 4, 1, 2, false, false, kVarGroupIssuesMma>(m, p, s.ctas, st, pdl);
         break;
     }
+  } else if (pair) {
+    e = launch_pair(Xq, M, K, m, p, s.ctas, st, pdl);
   } else {
     switch (variant) {
       case W4A8_VARIANT_BASELINE: e = launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl); break;

@@ -184,6 +184,13 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
  *                     previous one (no overlap of the two)
  *   GROUP_ISSUES_MMA  one dequantization warpgroup that also issues the MMAs
  *                     (no dedicated MMA warp)
+ *   CTA_PAIR          the 256-token tile computed by a pair of CTAs with
+ *                     CTA-pair MMAs (tcgen05 cta_group::2): each CTA holds
+ *                     its 128 channels and loads half of the tokens, with an
+ *                     8-deep ring; no split-K.  Needs M >= 256 and an even
+ *                     number of 128-channel blocks (else
+ *                     W4A8_ERR_UNSUPPORTED_SHAPE).  The default uses this
+ *                     form wherever it applies.
  * DEFAULT is the library's own choice (w4a8_gemm_ex / w4a8_gemm_i32).
  * Exactly one of Y (bf16, with s_x) or acc (INT32) is non-NULL.  Other
  * arguments as for w4a8_gemm_ex.
@@ -194,6 +201,7 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
 #define W4A8_VARIANT_SERIAL 3
 #define W4A8_VARIANT_ONE_GROUP 4
 #define W4A8_VARIANT_GROUP_ISSUES_MMA 5
+#define W4A8_VARIANT_CTA_PAIR 6
 
 int w4a8_gemm_variant(int variant, const int8_t* Xq, const float* s_x,
                       const void* packed, int M, int N, int K, uint16_t* Y,

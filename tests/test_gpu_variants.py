@@ -62,3 +62,50 @@ def test_variant_rejections():
     assert L.w4a8_gemm_variant(9, None, None, None, 0, 128, 256, None, None, 0, st) == w4.ERR_INVALID_ARG
     x = torch.zeros(4, dtype=torch.int32, device="cuda")
     assert L.w4a8_gemm_variant(1, None, None, None, 1, 128, 256, x.data_ptr(), x.data_ptr(), 0, st) == w4.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("M,N,K,kind", [(256, 256, 512, "normal"),     # one CTA pair
+                                        (512, 512, 1024, "heavy"),     # 2 token tiles x 2 pairs
+                                        (1000, 256, 2048, "ties"),     # ragged last token tile
+                                        (256, 1024, 128, "normal")])   # one k tile
+def test_cta_pair_variant_parity(M, N, K, kind):
+    pk, Xq, sx, acc_ref, y_ref = _case(M, N, K, kind)
+    acc = w4.w4a8_gemm_variant("cta_pair", Xq, None, pk, i32=True)
+    Y = w4.w4a8_gemm_variant("cta_pair", Xq, sx, pk, flags=w4.W4A8_FLAG_PDL)
+    torch.cuda.synchronize()
+    assert w4.w4a8_get_status() == 0
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_bf16_within_1ulp(bf16_bits(Y), y_ref, "cta_pair M=%d" % M)
+
+
+def test_cta_pair_needs_even_channel_blocks():
+    pk, Xq, sx, _, _ = _case(256, 384, 256, "normal")   # 3 channel blocks
+    with pytest.raises(w4.W4A8Error) as e:
+        w4.w4a8_gemm_variant("cta_pair", Xq, sx, pk)
+    assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
+
+
+def test_default_path_takes_the_cta_pair_at_large_m():
+    """A prefill-like shape runs the pair form by default (splits 1, 256-token
+    tiles, even channel blocks) and matches the oracle."""
+    M, N, K = 2048, 2048, 1024
+    assert w4.w4a8_gemm_schedule(M, N, K)[:2] == (256, 1)
+    pk, Xq, sx, acc_ref, y_ref = _case(M, N, K, "normal")
+    acc = w4.w4a8_gemm_i32(Xq, pk)
+    Y = w4.w4a8_gemm(Xq, sx, pk)
+    torch.cuda.synchronize()
+    assert w4.w4a8_get_status() == 0
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_bf16_within_1ulp(bf16_bits(Y), y_ref, "default pair")
+
+
+def test_cta_pair_repeated_runs_are_identical():
+    """The pair's cross-CTA hand-off (the odd CTA's weight slots and token
+    half feed the even CTA's MMAs) gives the same bits run after run."""
+    M, N, K = 1024, 1024, 4096
+    pk, Xq, sx, acc_ref, _ = _case(M, N, K, "normal")
+    for _ in range(6):
+        acc = w4.w4a8_gemm_variant("cta_pair", Xq, None, pk, i32=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert w4.w4a8_get_status() == 0
