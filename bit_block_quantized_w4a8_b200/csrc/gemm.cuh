@@ -169,12 +169,20 @@ __device__ __forceinline__ void dequant_chunk_naive(uint4 v, int s, int mn, uint
   }
 }
 
+constexpr int kClusterMax = 8;  // largest split-K cluster (portable cluster size)
+
 // Kernel variants for the ablation study (the production kernel is 0).
 enum : int {
   kVarDefault = 0,
   kVarNaiveDequant = 1,  // dequant_chunk_naive instead of IMAD + XOR
   kVarGroupIssuesMma = 2,  // the dequantization warpgroup issues the MMAs itself
 };
+
+// Two bf16 values (round to nearest even) packed low-first into 32 bits.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
 
 // One output: bf16(acc * (s_x * s_w)) in fp32 with a single rounding, or
 // the exact INT32 accumulator.
@@ -316,9 +324,13 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       }
       mbar_init(bar_acc, 1);
       mbar_init(bar_done, 4 * DQG);
-      mbar_init(bar_red, p.splits > 1 ? (uint32_t)(p.splits - 1) * 4 * DQG : 1u);
+      mbar_init(bar_red, 1);
       *abort_flag = 0;
       fence_barrier_init();
+      // push reduction: the leader's receive barrier completes when every
+      // other split's partial (t_valid x 128 INT32 adds) has landed
+      if (push && split == 0)
+        mbar_arrive_expect_tx(bar_red, (uint32_t)(p.splits - 1) * (uint32_t)t_valid * kTileN * 4u);
       pdl_launch_dependents();
     }
     __syncwarp();
@@ -616,22 +628,29 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       cluster_wait();
       const uint32_t red = sbase + C::kOffRed;
       if (split != 0) {
-        if (*ep_flag) {
-          const uint32_t red0 = dsmem_map(red, 0);
-          for (int j = dg; j < T / 16; j += DQG) {
-            if (16 * j >= t_valid) break;
-            uint32_t v[16];
+        // Every byte the leader expects is sent, zeros after an abort, so
+        // the leader's wait always ends and it never leaves while adds are
+        // still landing in its shared memory.
+        const uint32_t red0 = dsmem_map(red, 0);
+        const uint32_t bar0 = dsmem_map(bar_red, 0);
+        const bool live = *ep_flag != 0;  // uniform over the CTA
+        for (int j = dg; j < T / 16; j += DQG) {
+          if (16 * j >= t_valid) break;
+          uint32_t v[16];
+          if (live) {
             tmem_ld_x16(lane_base + 16 * j, v);
             tmem_wait_ld();
+          } else {
 #pragma unroll
-            for (int t = 0; t < 16; ++t)
-              if (16 * j + t < t_valid)
-                dsmem_red_add_s32(red0 + 4u * (uint32_t)((16 * j + t) * kTileN + r),
-                                  (int32_t)v[t]);
+            for (int t = 0; t < 16; ++t) v[t] = 0;
           }
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (16 * j + t < t_valid)
+              dsmem_red_async_add_s32(red0 + 4u * (uint32_t)((16 * j + t) * kTileN + r),
+                                      (int32_t)v[t], bar0);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(dsmem_map(bar_red, 0));  // also after an abort
       } else {
         warp_wait<true>(bar_red, 0, abort_flag, lim);  // remote arrivals: cluster scope
         if (*ep_flag) {
@@ -668,26 +687,38 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       const int per = ((total + p.splits - 1) / p.splits + 3) & ~3;
       const int e0 = split * per, e1 = min(total, e0 + per);
       const uint32_t part0 = sbase;
+      // whole-group vector stores when every output row starts 16 bytes
+      // aligned (N a multiple of 4 for bf16 8-byte stores, of 4 for INT32
+      // 16-byte stores) and the buffer itself is aligned
+      const bool vec_out = (p.N % 4) == 0 &&
+                           (p.Y ? (reinterpret_cast<uintptr_t>(p.Y) & 7) == 0
+                                : (reinterpret_cast<uintptr_t>(p.acc) & 15) == 0);
       constexpr int kBatch = 2;  // groups in flight per thread and round
       for (int eb = e0 + 4 * et; eb < e1; eb += 4 * nthr * kBatch) {
-        int4 acc4[kBatch];
+        // issue every remote load of the round (all splits) before using
+        // any of them: the loads are in flight together, not one round trip
+        // per split
+        int4 got[kClusterMax][kBatch];
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) acc4[b] = make_int4(0, 0, 0, 0);
-        // issue every remote load of the round before using any of them
-        for (int q = 0; q < p.splits; ++q) {
-          int4 got[kBatch];
+        for (int q = 0; q < kClusterMax; ++q) {
 #pragma unroll
           for (int b = 0; b < kBatch; ++b) {
             const int e = eb + 4 * nthr * b;
-            got[b] = e < e1 ? dsmem_ld_v4(dsmem_map(part0 + 4u * (uint32_t)e, (uint32_t)q))
+            got[q][b] = (q < p.splits && e < e1)
+                            ? dsmem_ld_v4(dsmem_map(part0 + 4u * (uint32_t)e, (uint32_t)q))
                             : make_int4(0, 0, 0, 0);
           }
+        }
+        int4 acc4[kBatch];
 #pragma unroll
-          for (int b = 0; b < kBatch; ++b) {
-            acc4[b].x += got[b].x;
-            acc4[b].y += got[b].y;
-            acc4[b].z += got[b].z;
-            acc4[b].w += got[b].w;
+        for (int b = 0; b < kBatch; ++b) {
+          acc4[b] = got[0][b];
+#pragma unroll
+          for (int q = 1; q < kClusterMax; ++q) {
+            acc4[b].x += got[q][b].x;
+            acc4[b].y += got[q][b].y;
+            acc4[b].z += got[q][b].z;
+            acc4[b].w += got[q][b].w;
           }
         }
 #pragma unroll
@@ -711,9 +742,23 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
           }
           const int32_t av[4] = {acc4[b].x, acc4[b].y, acc4[b].z, acc4[b].w};
           const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
+          const size_t o = (size_t)(row_base + t) * p.N + n2;
+          if (vec_out && n2 + 4 <= p.N) {
+            // the group's 4 channels are contiguous in the output row
+            if (p.Y) {
+              const float sx = sx_s[t];
+              uint2 w;
+              w.x = pack_bf16x2((float)av[0] * (sx * swv[0]), (float)av[1] * (sx * swv[1]));
+              w.y = pack_bf16x2((float)av[2] * (sx * swv[2]), (float)av[3] * (sx * swv[3]));
+              *reinterpret_cast<uint2*>(p.Y + o) = w;
+            } else {
+              *reinterpret_cast<int4*>(p.acc + o) = acc4[b];
+            }
+          } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (n2 + i < p.N) store_out(p, row_base + t, n2 + i, av[i], sx_s[t], swv[i]);
+            for (int i = 0; i < 4; ++i)
+              if (n2 + i < p.N) store_out(p, row_base + t, n2 + i, av[i], sx_s[t], swv[i]);
+          }
         }
       }
     }

@@ -380,6 +380,18 @@ __device__ __forceinline__ void dsmem_red_add_s32(uint32_t caddr, int32_t v) {
                : "memory");
 }
 
+// Asynchronous atomic add into another CTA's shared memory whose completion
+// is counted (4 bytes) on an mbarrier in that CTA: the receiver expects the
+// total bytes and waits for the phase, with no fence or arrival by the
+// sender.
+__device__ __forceinline__ void dsmem_red_async_add_s32(uint32_t caddr, int32_t v,
+                                                        uint32_t cbar) {
+  asm volatile(
+      "red.async.relaxed.cluster.shared::cluster.mbarrier::complete_tx::bytes.add.s32 "
+      "[%0], %1, [%2];" ::"r"(caddr), "r"(v), "r"(cbar)
+      : "memory");
+}
+
 // Arrive on an mbarrier in another CTA of the cluster; release at cluster
 // scope orders this thread's earlier shared::cluster writes before it.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
