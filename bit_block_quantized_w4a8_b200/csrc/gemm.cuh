@@ -64,7 +64,12 @@ struct GemmParams {
   int kt_total;           // K / 128
   int splits, kt_per_split;
   int n_tiles, m_tiles;
-  uint32_t x_tx_bytes;    // bytes of one activation box (rows * 128)
+  // Tokens per tile actually used (the MMA's N): T, or in the runtime-width
+  // instantiations of the 256-token tile a multiple of 16 below it (of 32
+  // for CTA pairs) sized to the rows, so that no MMA work goes to rows that
+  // do not exist.  The activation box is min(M, tn) rows (tn / 2 per CTA of
+  // a pair).
+  int tn;
   unsigned long long wait_limit_ns;
   const PackedHeader* hdr;  // checked against (N, K) before any store
   // Grouped GEMM (mixture-of-experts): rows [offsets[g], offsets[g+1]) of
@@ -83,6 +88,8 @@ struct GemmParams {
   // with evict-first), or reused by several (normal priority).
   int w_stream;
 };
+// (128 bytes: one more field measured 7% slower CTA-pair prefill launches)
+static_assert(sizeof(GemmParams) <= 128, "kernel parameter block");
 
 template <int T, int SS, int AS, int DQG, bool PUSH = false, bool W8 = false,
           bool PAIR = false>
@@ -205,12 +212,17 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8, int V, bool PAIR>
+template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8, int V, bool PAIR,
+          bool RTN>
 __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThreads, MINB)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_w,  // W8 only
                      const GemmParams p) {
   using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
+  // tokens per tile (MMA N): p.tn in the runtime-width instantiations,
+  // else the compile-time T (which keeps the full-tile code as tight as it
+  // was; a runtime width measured up to 20% slower on full tiles)
+  const int TN = RTN ? p.tn : T;
   static_assert(V != kVarGroupIssuesMma || (DQG == 1 && !W8),
                 "the issuing warpgroup must see every k tile");
   extern __shared__ uint8_t smem_raw[];
@@ -263,8 +275,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
   const float* w_scale = p.s_w;
   const PackedHeader* w_hdr = p.hdr;
   if (p.offsets == nullptr) {
-    row_base = m_slot * T;
-    t_valid = min(T, p.M - row_base);
+    row_base = m_slot * TN;
+    t_valid = min(TN, p.M - row_base);
   } else {
     // Grouped: the row offsets may be written by the preceding kernel.  Token
     // tile slot `a` is the a-th tile that holds rows, counting group by
@@ -282,7 +294,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
         bad = true;
         break;
       }
-      const int cnt = (q1 - q0 + T - 1) / T;
+      const int cnt = (q1 - q0 + TN - 1) / TN;
       if (g < 0) {
         if (a < cnt) {
           g = q;
@@ -299,8 +311,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       return;
     }
     if (g < 0) return;
-    row_base = r0 + m_tile * T;
-    t_valid = min(T, r1 - row_base);
+    row_base = r0 + m_tile * TN;
+    t_valid = min(TN, r1 - row_base);
     w_tiles += p.group_bytes * g;
     w_scale = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(w_scale) +
                                              p.group_bytes * g);
@@ -375,7 +387,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     // copies (a converged warp issues these single-thread instructions much
     // faster than a lone diverged lane).
     const bool leader = elect_one();
-    const uint32_t tx = C::kWBytes + p.x_tx_bytes;
+    // bytes of one stage: the weight tile and the activation box
+    const uint32_t tx = C::kWBytes + (uint32_t)(PAIR ? TN / 2 : min(p.M, TN)) * kTileK;
     if (leader) {
       prefetch_tensormap(&tmap_x);
       if (W8) prefetch_tensormap(&tmap_w);
@@ -407,7 +420,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     if (leader) {
       for (int it = 0; it < pre; ++it)
         tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
-                    row_base + rank * (T / 2), bar_full + 8 * it);
+                    row_base + rank * (TN / 2), bar_full + 8 * it);
     }
     issued = pre;
     __syncwarp();
@@ -419,7 +432,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
         mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         load_w(it, s);
         tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
-                    row_base + rank * (T / 2), bar_full + 8 * s);
+                    row_base + rank * (TN / 2), bar_full + 8 * s);
       }
       __syncwarp();
       issued = it + 1;
@@ -442,7 +455,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     // fence off the dequantization warps.
     if (rank == 0) {
       const bool leader = elect_one();
-      constexpr uint32_t idesc = idesc_i8(256, T);
+      const uint32_t idesc = idesc_i8(256, TN);
       for (int it = 0; it < nk; ++it) {
         const int s = it % SS, a = it % AS;
         if (!warp_wait<true>(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
@@ -467,7 +480,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     // ---------------------------------------------------------- MMA issuer
     // Whole warp waits, one elected lane issues the MMAs and commits.
     const bool leader = elect_one();
-    constexpr uint32_t idesc = idesc_i8(128, T);
+    const uint32_t idesc = idesc_i8(128, TN);
     for (int it = 0; it < nk; ++it) {
       const int s = it % SS, a = it % AS;
       if (!W8 && !warp_wait(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
@@ -562,7 +575,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
           const uint32_t a_tmem = tmem + C::kA0 + 32 * a;
 #pragma unroll
           for (int kk = 0; kk < kTileK / 32; ++kk)
-            mma_i8_ts(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc_i8(128, T),
+            mma_i8_ts(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc_i8(128, TN),
                       (it | kk) != 0);
           tc_commit(bar_empty + 8 * s);
           tc_commit(bar_afree + 8 * a);

@@ -100,13 +100,13 @@ bool make_w8_map(CUtensorMap* map, const int8_t* Wq, int N, int K) {
 
 // -------------------------------------------------- kernel attributes
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
-          int V = kVarDefault, bool PAIR = false>
+          int V = kVarDefault, bool PAIR = false, bool RTN = false>
 cudaError_t ensure_smem_attr() {
   using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
-    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR>,
+    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -274,12 +274,12 @@ struct Maps {
 };
 
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
-          int V = kVarDefault, bool PAIR = false>
+          int V = kVarDefault, bool PAIR = false, bool RTN = false>
 cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream_t st,
                         bool pdl) {
   using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
-  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR>;
-  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR>();
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN>;
+  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN>();
   if (ea != cudaSuccess) return ea;
   return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl,
                   PAIR ? 2 : p.splits, m.x, m.w, p);
@@ -302,9 +302,12 @@ bool use_pair(const Schedule& s, int M) {
 // Pair launch: the activation box is the CTA's half of the token tile.
 cudaError_t launch_pair(const int8_t* Xq, int M, int K, Maps& m, GemmParams& p, int ctas,
                         cudaStream_t st, bool pdl) {
-  if (!make_act_map(&m.x, Xq, M, K, 128)) return cudaErrorInvalidValue;
-  p.x_tx_bytes = 128u * kTileK;
-  return launch_gemm<256, 8, 4, 2, 1, false, false, kVarDefault, true>(m, p, ctas, st, pdl);
+  p.tn = round_up(p.tn, 32);  // each CTA loads tn / 2 rows
+  if (!make_act_map(&m.x, Xq, M, K, p.tn / 2)) return cudaErrorInvalidValue;
+  return p.tn == 256
+             ? launch_gemm<256, 8, 4, 2, 1, false, false, kVarDefault, true>(m, p, ctas, st, pdl)
+             : launch_gemm<256, 8, 4, 2, 1, false, false, kVarDefault, true, true>(m, p, ctas, st,
+                                                                                   pdl);
 }
 
 // Checks shared by both weight formats; fills the launch-independent part
@@ -321,6 +324,11 @@ int check_common(const int8_t* Xq, const float* s_x, const void* w, int M, int N
     return W4A8_ERR_MISALIGNED;
   return W4A8_OK;
 }
+
+// Activation box of a single-CTA tile: only rows that exist are fetched when
+// M < tn (the MMA still reads tn rows, but rows past M only feed accumulator
+// columns that are never stored).  The kernel expects exactly these bytes.
+int box_rows(const GemmParams& p) { return p.M < p.tn ? p.M : p.tn; }
 
 GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K, uint16_t* Y,
                        int32_t* acc) {
@@ -351,10 +359,10 @@ GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K,
   // streamed with an evict-first hint.
   p.m_band = s.m_tiles < kRasterBand ? s.m_tiles : kRasterBand;
   p.w_stream = s.m_tiles == 1 ? 1 : 0;
-  // Only rows that exist are fetched when M < T: the MMA still reads T rows,
-  // but rows past M only feed accumulator columns that are never stored.
-  const int box_rows = M < s.T ? M : s.T;
-  p.x_tx_bytes = (uint32_t)box_rows * kTileK;
+  // The 256-token configurations size the tile to the rows: the token tiles
+  // share M evenly, rounded up to the MMA's granularity of 16.
+  p.tn = s.T;
+  if (s.T == 256 && s.m_tiles > 0) p.tn = round_up((M + s.m_tiles - 1) / s.m_tiles, 16);
   return p;
 }
 
@@ -390,13 +398,15 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     p.m_total = g.m_total;
     p.groups = g.groups;
     p.m_band = 1;
-    p.w_stream = M <= s.T ? 1 : 0;  // one token tile per group
+    // groups of up to 256 rows take one tile of their bound's width
+    if (s.T == 256) p.tn = round_up(M < 256 ? M : 256, 16);
+    p.w_stream = M <= p.tn ? 1 : 0;  // one token tile per group
   }
 
   Maps m;
   // the box holds min(T, M) rows: every valid row of a tile (grouped: M
-  // bounds each group's rows), and exactly the bytes x_tx_bytes expects
-  if (!make_act_map(&m.x, Xq, x_rows, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
+  // bounds each group's rows), and exactly the bytes the kernel expects
+  if (!make_act_map(&m.x, Xq, x_rows, K, box_rows(p))) return W4A8_ERR_CUDA;
   m.w = m.x;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
@@ -421,9 +431,13 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     case 64: e = launch_gemm<64, 6, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 4, 4, 2, 2>(m, p, s.ctas, st, pdl); break;  // tuning only
     default:
-      e = (g.groups == 0 && use_pair(s, M))
-              ? launch_pair(Xq, M, K, m, p, s.ctas, st, pdl)
-              : launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl);
+      if (g.groups == 0 && use_pair(s, M))
+        e = launch_pair(Xq, M, K, m, p, s.ctas, st, pdl);
+      else if (p.tn == 256)
+        e = launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl);
+      else
+        e = launch_gemm<256, 5, 4, 2, 1, false, false, kVarDefault, false, true>(m, p, s.ctas,
+                                                                                st, pdl);
       break;
   }
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
@@ -445,9 +459,10 @@ int gemm_w8_common(const int8_t* Xq, const float* s_x, const int8_t* Wq, const f
   const Schedule s = choose_schedule(M, N, K, num_sms(dev), true);
   GemmParams p = make_params(s, s_x, M, N, K, Y, acc);
   p.s_w = s_w;
+  p.tn = s.T;  // the W8A8 kernel keeps whole tiles
 
   Maps m;
-  if (!make_act_map(&m.x, Xq, M, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
+  if (!make_act_map(&m.x, Xq, M, K, box_rows(p))) return W4A8_ERR_CUDA;
   if (!make_w8_map(&m.w, Wq, N, K)) return W4A8_ERR_CUDA;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
@@ -488,12 +503,15 @@ int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* pa
     return W4A8_ERR_UNSUPPORTED_SHAPE;
   const Schedule s = choose_schedule(M, N, K, num_sms(dev), false, 0, T, pair ? 1 : 0);
   GemmParams p = make_params(s, s_x, M, N, K, Y, acc);
+  if (!pair) {
+    p.tn = s.T;  // the ablation variants keep whole tiles
+    }
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   p.tiles = base + tiles_offset_bytes(p.n_pad);
   p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
   p.hdr = reinterpret_cast<const PackedHeader*>(base);
   Maps m;
-  if (!make_act_map(&m.x, Xq, M, K, M < s.T ? M : s.T)) return W4A8_ERR_CUDA;
+  if (!make_act_map(&m.x, Xq, M, K, box_rows(p))) return W4A8_ERR_CUDA;
   m.w = m.x;
   cudaStream_t st = as_stream(stream);
   cudaError_t e = cudaErrorInvalidValue;
