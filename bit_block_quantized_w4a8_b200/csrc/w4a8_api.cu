@@ -289,14 +289,17 @@ cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream
 // each holds 128 channels and loads half of the tokens, so a stage is
 // 16 KB of activations instead of 32 KB and the ring is 8 deep instead of
 // 5): taken for dense calls without split-K whose channel blocks pair up
-// and whose token tiles are full height.  W4A8_PAIR=0 in the environment
-// turns it off (tuning only).
-bool use_pair(const Schedule& s, int M) {
+// and whose token tiles are full height.  (Grouped calls keep the
+// single-CTA tile: on the Mixtral-like prefill the pair was 5% slower for
+// the wide layer and 2% faster for the narrow one.)  W4A8_PAIR=0 in the
+// environment turns it off (tuning only).
+bool use_pair(const Schedule& s, const GemmParams& p, bool grouped) {
   static const bool enabled = [] {
     const char* v = getenv("W4A8_PAIR");
     return !(v && v[0] == '0');
   }();
-  return enabled && s.T == 256 && s.splits == 1 && s.n_tiles % 2 == 0 && M >= 256;
+  return enabled && !grouped && s.T == 256 && s.splits == 1 && s.n_tiles % 2 == 0 &&
+         p.M >= 256;
 }
 
 // Pair launch: the activation box is the CTA's half of the token tile.
@@ -431,8 +434,8 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     case 64: e = launch_gemm<64, 6, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 4, 4, 2, 2>(m, p, s.ctas, st, pdl); break;  // tuning only
     default:
-      if (g.groups == 0 && use_pair(s, M))
-        e = launch_pair(Xq, M, K, m, p, s.ctas, st, pdl);
+      if (use_pair(s, p, g.groups > 0))
+        e = launch_pair(Xq, x_rows, K, m, p, s.ctas, st, pdl);
       else if (p.tn == 256)
         e = launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl);
       else

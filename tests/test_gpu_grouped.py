@@ -53,6 +53,7 @@ CASES = [
     ([10, 10, 10], 200, 384),                  # ragged N
     ([0, 0, 7], 128, 128),                     # only the last expert has rows
     ([33], 256, 256),                          # one group = a dense GEMM
+    ([150, 90, 0, 200], 4096, 1024),           # 208-token tiles (runtime width), no split
 ]
 
 
@@ -160,3 +161,10 @@ def test_mixtral_like_full_size(layer_name, tokens):
             W8 = oracle.dequant_weights(wqs[e]["codes"], wqs[e]["s_u8"], wqs[e]["a"])
             colsum = W8.sum(axis=0, dtype=np.int64)
             assert np.array_equal(rows[o[e]:o[e + 1]], Xq_ref[o[e]:o[e + 1]].astype(np.int64) @ colsum)
+
+
+def test_grouped_prefill_shape_uses_the_wide_tile():
+    """The case above runs without split-K on the 256-token configuration,
+    its tile width sized to the largest group."""
+    T, splits, _ = w4.w4a8_grouped_gemm_schedule(4, 440, 200, 4096, 1024)
+    assert (T, splits) == (256, 1)
