@@ -141,6 +141,16 @@ bool light16_enabled() {
   return ok;
 }
 
+// The CTA-pair form of the 256-token tile (see use_pair below).
+// W4A8_PAIR=0 in the environment turns it off (tuning only).
+bool pair_enabled() {
+  static const bool enabled = [] {
+    const char* v = getenv("W4A8_PAIR");
+    return !(v && v[0] == '0');
+  }();
+  return enabled;
+}
+
 // CTAs of one configuration that fit on an SM at once (shared memory and
 // TMEM permitting); matches the MINB column of the launch tables below.
 int ctas_per_sm(int T, int kt_per, bool w8) {
@@ -164,7 +174,11 @@ int ctas_per_sm(int T, int kt_per, bool w8) {
 //   per k tile through a shallower ring (bytes in flight per CTA bound it:
 //   0.35..0.45 us per k tile);
 // - the cluster reduction costs ~0.1 us per halving step plus, for the
-//   gather form, the partial tile (0.005 us per token column).
+//   gather form, the partial tile (0.005 us per token column);
+// - without split-K a dense call of full 256-token tiles with paired
+//   channel blocks runs the CTA-pair form, whose deeper ring takes 0.22 us
+//   per k tile instead of 0.29 (measured: one split then beats two on the
+//   70B-like layers at M = 384..2048, and loses on the 4096-wide ones).
 // Ties go to more splits.  W4A8_FORCE_SPLITS=<n> and W4A8_FORCE_TILE=<tokens>
 // in the environment override the choice (tuning only).
 Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_tiles = 0,
@@ -193,6 +207,8 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_ti
     const char* e = getenv("W4A8_FORCE_SPLITS");
     return e ? atoi(e) : 0;
   }();
+  const bool pair_ok = pair_enabled() && !w8 && active_m_tiles == 0 && s.T == 256 &&
+                       s.n_tiles % 2 == 0 && M >= 256;
   double best = 1e300;
   for (int cand = 1; cand <= kMaxSplits && cand <= kt; ++cand) {
     const int per = (kt + cand - 1) / cand;
@@ -204,7 +220,8 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_ti
     const long waves = (tiles + per_wave - 1) / per_wave;
     const long resident = (tiles < per_wave ? tiles : per_wave) * eff;
     const double t_bw = resident * w_bytes / kBytesPerUs;
-    const double t_tile = t_cta > t_bw ? t_cta : t_bw;
+    const double t_own = (pair_ok && eff == 1) ? 0.22 : t_cta;
+    const double t_tile = t_own > t_bw ? t_own : t_bw;
     const int lg = eff > 4 ? 3 : eff > 2 ? 2 : eff > 1 ? 1 : 0;
     const double tok = M < s.T ? M : s.T;
     const double red = lg * (0.1 + (push ? 0.05 : 0.005 * tok));
@@ -291,14 +308,9 @@ cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream
 // 5): taken for dense calls without split-K whose channel blocks pair up
 // and whose token tiles are full height.  (Grouped calls keep the
 // single-CTA tile: on the Mixtral-like prefill the pair was 5% slower for
-// the wide layer and 2% faster for the narrow one.)  W4A8_PAIR=0 in the
-// environment turns it off (tuning only).
+// the wide layer and 2% faster for the narrow one.)
 bool use_pair(const Schedule& s, const GemmParams& p, bool grouped) {
-  static const bool enabled = [] {
-    const char* v = getenv("W4A8_PAIR");
-    return !(v && v[0] == '0');
-  }();
-  return enabled && !grouped && s.T == 256 && s.splits == 1 && s.n_tiles % 2 == 0 &&
+  return pair_enabled() && !grouped && s.T == 256 && s.splits == 1 && s.n_tiles % 2 == 0 &&
          p.M >= 256;
 }
 

@@ -67,7 +67,9 @@ def test_variant_rejections():
 @pytest.mark.parametrize("M,N,K,kind", [(256, 256, 512, "normal"),     # one CTA pair
                                         (512, 512, 1024, "heavy"),     # 2 token tiles x 2 pairs
                                         (1000, 256, 2048, "ties"),     # ragged last token tile
-                                        (256, 1024, 128, "normal")])   # one k tile
+                                        (256, 1024, 128, "normal"),    # one k tile
+                                        (300, 512, 1024, "normal"),    # 2 tiles of 160 (runtime width)
+                                        (600, 256, 512, "heavy")])     # 3 tiles of 224 (runtime width)
 def test_cta_pair_variant_parity(M, N, K, kind):
     pk, Xq, sx, acc_ref, y_ref = _case(M, N, K, kind)
     acc = w4.w4a8_gemm_variant("cta_pair", Xq, None, pk, i32=True)
