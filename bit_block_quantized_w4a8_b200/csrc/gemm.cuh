@@ -54,6 +54,8 @@
 
 namespace w4a8 {
 
+enum : int { kModeStreamW = 1, kModeStoreY = 2 };
+
 struct GemmParams {
   const uint8_t* tiles;   // packed weight tiles
   const float* s_w;       // packed per-channel scales [n_pad]
@@ -84,9 +86,11 @@ struct GemmParams {
   // block by channel block, so that a wave of CTAs reuses both operands in
   // L2 (1 = channel blocks first).
   int m_band;
-  // Weight tiles are read by one token tile only (stream them through L2
-  // with evict-first), or reused by several (normal priority).
-  int w_stream;
+  // kModeStreamW: weight tiles are read by one token tile only (stream them
+  // through L2 with evict-first; else normal priority).
+  // kModeStoreY: without split-K, the bf16 tile is staged in shared memory
+  // and written by one TMA tensor store through the second tensor map.
+  int mode;
 };
 // (128 bytes: one more field measured 7% slower CTA-pair prefill launches)
 static_assert(sizeof(GemmParams) <= 128, "kernel parameter block");
@@ -391,9 +395,10 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     const uint32_t tx = C::kWBytes + (uint32_t)(PAIR ? TN / 2 : min(p.M, TN)) * kTileK;
     if (leader) {
       prefetch_tensormap(&tmap_x);
-      if (W8) prefetch_tensormap(&tmap_w);
+      if (W8 || (p.mode & kModeStoreY)) prefetch_tensormap(&tmap_w);
     }
-    const uint64_t pol = p.w_stream ? l2_policy_evict_first() : l2_policy_evict_normal();
+    const uint64_t pol =
+        (p.mode & kModeStreamW) ? l2_policy_evict_first() : l2_policy_evict_normal();
     const uint8_t* wsrc = W8 ? nullptr
                              : w_tiles + ((size_t)n_tile * p.kt_total + kt0) * kTileBytes;
     // one weight stage: a bulk copy of the packed tile, or a TMA box of
@@ -607,7 +612,32 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     __syncwarp();
     named_bar_sync(1, nthr);
     if (*ep_flag) {
-      if (p.splits == 1) {
+      if (!W8 && p.splits == 1 && (p.mode & kModeStoreY)) {
+        // stage the bf16 tile as [token][128 channels] in the (free) stage
+        // buffers, then one thread writes it with a TMA tensor store; rows
+        // past M and channels past N are clipped by the store
+        const uint32_t ystage = sbase;
+        for (int j = dg; j < T / 16; j += DQG) {
+          uint32_t v[16];
+          tmem_ld_x16(lane_base + 16 * j, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int tt = 16 * j + t;
+            const float y = (float)(int32_t)v[t] * (sx_s[tt] * swn);
+            sts16(ystage + (uint32_t)(tt * kTileN + r) * 2u,
+                  __bfloat16_as_ushort(__float2bfloat16_rn(y)));
+          }
+        }
+        fence_proxy_async_smem();  // the stores above, seen by the TMA engine
+        named_bar_sync(1, nthr);
+        if (threadIdx.x == 64) {
+          tma_store_2d(&tmap_w, n_tile * kTileN, row_base, ystage);
+          bulk_commit_group();
+          bulk_wait_group_all();
+        }
+        __syncwarp();
+      } else if (p.splits == 1) {
         for (int j = dg; j < T / 16; j += DQG) {
           uint32_t v[16];
           tmem_ld_x16(lane_base + 16 * j, v);

@@ -81,6 +81,23 @@ bool make_act_map(CUtensorMap* map, const int8_t* Xq, int M, int K, int rows) {
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over the bf16 output Y [M][N] (N contiguous) for the TMA store
+// of a tile: boxes of 128 channels by `rows` tokens, no swizzle; the store
+// leaves elements outside [M, N] alone.  Needs N a multiple of 8 (16-byte
+// row stride) and Y 16-byte aligned.
+bool make_y_map(CUtensorMap* map, uint16_t* Y, int M, int N, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kTileN, (cuuint32_t)rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, Y, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Tensor map over INT8 weights Wq [N][K] (K contiguous), for the W8A8
 // comparison kernel: boxes of 128 bytes of k by 128 channels, 128-byte
 // swizzle (the MMA's K-major operand layout), zero fill past channel N.
@@ -309,6 +326,16 @@ cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream
 // and whose token tiles are full height.  (Grouped calls keep the
 // single-CTA tile: on the Mixtral-like prefill the pair was 5% slower for
 // the wide layer and 2% faster for the narrow one.)
+// Bf16 tiles written by a TMA store from shared memory (dense calls without
+// split-K).  W4A8_STORE_Y=0 in the environment turns it off (tuning only).
+bool store_y_enabled() {
+  static const bool enabled = [] {
+    const char* v = getenv("W4A8_STORE_Y");
+    return !(v && v[0] == '0');
+  }();
+  return enabled;
+}
+
 bool use_pair(const Schedule& s, const GemmParams& p, bool grouped) {
   return pair_enabled() && !grouped && s.T == 256 && s.splits == 1 && s.n_tiles % 2 == 0 &&
          p.M >= 256;
@@ -373,7 +400,7 @@ GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K,
   // L2 while the wave reuses them.  Weights read by one token tile only are
   // streamed with an evict-first hint.
   p.m_band = s.m_tiles < kRasterBand ? s.m_tiles : kRasterBand;
-  p.w_stream = s.m_tiles == 1 ? 1 : 0;
+  p.mode = s.m_tiles == 1 ? kModeStreamW : 0;
   // The 256-token configurations size the tile to the rows: the token tiles
   // share M evenly, rounded up to the MMA's granularity of 16.
   p.tn = s.T;
@@ -415,14 +442,22 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     p.m_band = 1;
     // groups of up to 256 rows take one tile of their bound's width
     if (s.T == 256) p.tn = round_up(M < 256 ? M : 256, 16);
-    p.w_stream = M <= p.tn ? 1 : 0;  // one token tile per group
+    p.mode = M <= p.tn ? kModeStreamW : 0;  // one token tile per group
   }
+
+  const bool pair = s.T == 256 && use_pair(s, p, g.groups > 0);
+  if (pair) p.tn = round_up(p.tn, 32);  // each CTA of a pair loads tn / 2 rows
 
   Maps m;
   // the box holds min(T, M) rows: every valid row of a tile (grouped: M
   // bounds each group's rows), and exactly the bytes the kernel expects
   if (!make_act_map(&m.x, Xq, x_rows, K, box_rows(p))) return W4A8_ERR_CUDA;
   m.w = m.x;
+  // Dense calls without split-K write their bf16 tile with one TMA store
+  // (the second tensor map); the box is the CTA's tile rows.
+  if (g.groups == 0 && Y && s.splits == 1 && N % 8 == 0 && aligned(Y, 16) && store_y_enabled() &&
+      make_y_map(&m.w, Y, M, N, pair ? p.tn : box_rows(p)))
+    p.mode |= kModeStoreY;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
   switch (s.T) {
@@ -446,7 +481,7 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
     case 64: e = launch_gemm<64, 6, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 4, 4, 2, 2>(m, p, s.ctas, st, pdl); break;  // tuning only
     default:
-      if (use_pair(s, p, g.groups > 0))
+      if (pair)
         e = launch_pair(Xq, x_rows, K, m, p, s.ctas, st, pdl);
       else if (p.tn == 256)
         e = launch_gemm<256, 5, 4, 2, 1>(m, p, s.ctas, st, pdl);
