@@ -126,7 +126,9 @@ struct GemmCfg {
   static constexpr int kOffBar = kOffW + SS * kWBytes;
   static_assert(!W8 || (kOffW % 1024 == 0 && kWBytes % 1024 == 0),
                 "128-byte-swizzled operand tiles start on 1024-byte boundaries");
-  static constexpr int kNumBars = 2 * SS + 2 * AS + 3;
+  // stage barriers: weights landed, activations landed (not in the CTA-pair
+  // form, which lands both on one), stage free; slot barriers; 3 more
+  static constexpr int kNumBars = (PAIR ? 2 : 3) * SS + 2 * AS + 3;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffSx = kOffMisc + 16;
   // partial tiles of at most kPushMaxM tokens are pushed (remote atomic
@@ -235,8 +237,16 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // Each stage has two landing barriers, weights (bar_full) and activations
+  // (bar_fullx): the weight tiles are prefetched before the preceding
+  // kernel finishes, and their dequantization need not wait for the
+  // activations, which only the MMAs read (decode: 11-18% per quantize +
+  // GEMM pair).  The CTA-pair form (large M, nothing to prefetch early)
+  // lands both on bar_full, which measured 3% faster there.
+  constexpr bool kSplitLand = !PAIR;
   const uint32_t bar_full = sbase + C::kOffBar;     // + 8 ss
-  const uint32_t bar_empty = bar_full + 8 * SS;     // + 8 ss
+  const uint32_t bar_fullx = kSplitLand ? bar_full + 8 * SS : bar_full;  // + 8 ss
+  const uint32_t bar_empty = bar_full + (kSplitLand ? 16 : 8) * SS;  // + 8 ss
   const uint32_t bar_dq = bar_empty + 8 * SS;       // + 8 as
   const uint32_t bar_afree = bar_dq + 8 * AS;       // + 8 as
   const uint32_t bar_acc = bar_afree + 8 * AS;
@@ -331,6 +341,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     if (lane == 0) {
       for (int s = 0; s < SS; ++s) {
         mbar_init(bar_full + 8 * s, 1);
+        if (kSplitLand) mbar_init(bar_fullx + 8 * s, 1);
         mbar_init(bar_empty + 8 * s, 1);
       }
       for (int a = 0; a < AS; ++a) {
@@ -391,8 +402,11 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     // copies (a converged warp issues these single-thread instructions much
     // faster than a lone diverged lane).
     const bool leader = elect_one();
-    // bytes of one stage: the weight tile and the activation box
-    const uint32_t tx = C::kWBytes + (uint32_t)(PAIR ? TN / 2 : min(p.M, TN)) * kTileK;
+    // bytes landing on a stage's two barriers: the weight tile, and the
+    // activation box
+    const uint32_t x_bytes = (uint32_t)(PAIR ? TN / 2 : min(p.M, TN)) * kTileK;
+    const uint32_t tx_w = kSplitLand ? C::kWBytes : C::kWBytes + x_bytes;
+    const uint32_t tx_x = x_bytes;
     if (leader) {
       prefetch_tensormap(&tmap_x);
       if (W8 || (p.mode & kModeStoreY)) prefetch_tensormap(&tmap_w);
@@ -417,15 +431,17 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     const int pre = nk < SS ? nk : SS;
     if (leader) {
       for (int it = 0; it < pre; ++it) {
-        mbar_arrive_expect_tx(bar_full + 8 * it, tx);
+        mbar_arrive_expect_tx(bar_full + 8 * it, tx_w);
         load_w(it, it);
       }
     }
     pdl_wait();  // activations are produced by the preceding kernel
     if (leader) {
-      for (int it = 0; it < pre; ++it)
+      for (int it = 0; it < pre; ++it) {
+        if (kSplitLand) mbar_arrive_expect_tx(bar_fullx + 8 * it, tx_x);
         tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
-                    row_base + rank * (TN / 2), bar_full + 8 * it);
+                    row_base + rank * (TN / 2), bar_fullx + 8 * it);
+      }
     }
     issued = pre;
     __syncwarp();
@@ -434,18 +450,21 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       const uint32_t ph = (it / SS) & 1;
       if (!warp_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, lim)) break;
       if (leader) {
-        mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+        mbar_arrive_expect_tx(bar_full + 8 * s, tx_w);
         load_w(it, s);
+        if (kSplitLand) mbar_arrive_expect_tx(bar_fullx + 8 * s, tx_x);
         tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
-                    row_base + rank * (TN / 2), bar_full + 8 * s);
+                    row_base + rank * (TN / 2), bar_fullx + 8 * s);
       }
       __syncwarp();
       issued = it + 1;
     }
     if (*abort_flag) {
       // let the copies already issued land before the CTA goes away
-      for (int it = issued - SS < 0 ? 0 : issued - SS; it < issued; ++it)
+      for (int it = issued - SS < 0 ? 0 : issued - SS; it < issued; ++it) {
         mbar_wait(bar_full + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
+        if (kSplitLand) mbar_wait(bar_fullx + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
+      }
     }
     __syncwarp();  // reconverge before any CTA- or cluster-wide barrier
   } else if (warp == 1 && PAIR) {
@@ -464,7 +483,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       for (int it = 0; it < nk; ++it) {
         const int s = it % SS, a = it % AS;
         if (!warp_wait<true>(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
-        if (!warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
+        if (!warp_wait(bar_fullx + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
         tc_fence_after();
         if (leader) {
           const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
@@ -488,8 +507,11 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     const uint32_t idesc = idesc_i8(128, TN);
     for (int it = 0; it < nk; ++it) {
       const int s = it % SS, a = it % AS;
+      // the weights reach the MMA through the dequantized slot (dq), except
+      // in the W8A8 form, which reads the stage's INT8 weight tile directly
       if (!W8 && !warp_wait(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
-      if (!warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
+      if (W8 && !warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
+      if (!warp_wait(bar_fullx + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
       tc_fence_after();
       if (leader) {
         const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
@@ -539,6 +561,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       // before this one has landed, because AS <= SS.
       if (!warp_wait(bar_afree + 8 * a, ((it / AS) & 1) ^ 1, abort_flag, lim)) break;
       if (!warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
+      // (in the CTA-pair form bar_full also covers the token half, which the
+      // odd CTA's arrival on the even one's slot barrier thereby implies)
       tc_fence_after();
       // all shared-memory reads first (independent), then the arithmetic,
       // then one 32-column TMEM store of this row's 128 dequantized weights
@@ -574,6 +598,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
         // ablation: the first warp of the (single) dequantization group
         // issues this k tile's MMAs once all four quarters are in TMEM
         if (!warp_wait(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
+        if (!warp_wait(bar_fullx + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
         tc_fence_after();
         if (elect_one()) {
           const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
