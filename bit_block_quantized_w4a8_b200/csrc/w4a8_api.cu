@@ -182,7 +182,7 @@ int ctas_per_sm(int T, int kt_per, bool w8) {
 // - a wave is as many clusters (the splits of one output tile) as the SMs
 //   hold at once; a cluster whose size is not a power of two does not tile
 //   the SMs of a GPC evenly, so only 92% of the slots count for it;
-// - fill is launch, pipeline fill and epilogue (3.5 us for 16..64-token
+// - fill is launch, pipeline fill and epilogue (3 us for 16..64-token
 //   tiles, 7.4 us for the 256-token tile);
 // - t_tile is one k tile's time per CTA: the slower of the CTA's own
 //   dequantize + MMA chain (0.27 us for 16 tokens, 0.29 us for 256) and its
@@ -190,8 +190,9 @@ int ctas_per_sm(int T, int kt_per, bool w8) {
 //   6 TB/s sustained); the W8A8 comparison kernel reads 16 KB of weights
 //   per k tile through a shallower ring (bytes in flight per CTA bound it:
 //   0.35..0.45 us per k tile);
-// - the cluster reduction costs ~0.1 us per halving step plus, for the
-//   gather form, the partial tile (0.005 us per token column);
+// - the cluster reduction: the push form ~0.1 us per halving step; the
+//   gather form 0.2 us per split (two cluster barriers, remote reads from
+//   every split) plus the partial tile's width;
 // - without split-K a dense call of full 256-token tiles with paired
 //   channel blocks runs the CTA-pair form, whose deeper ring takes 0.22 us
 //   per k tile instead of 0.29 (measured: one split then beats two on the
@@ -214,9 +215,9 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_ti
   const int kt = K / kTileK;
   // tiles that do work (grouped GEMMs launch more, which leave at once)
   const long tiles = (long)s.n_tiles * (active_m_tiles > 0 ? active_m_tiles : s.m_tiles);
-  const double fill = s.T <= 64 ? (s.T == 16 ? 3.5 : 3.7) : s.T == 128 ? 6.0 : 7.4;
+  const double fill = s.T <= 64 ? 3.0 : s.T == 128 ? 6.0 : 7.4;
   const double t_cta = w8 ? (s.T == 16 ? 0.35 : s.T == 32 ? 0.40 : s.T == 64 ? 0.45 : 0.35)
-                         : (s.T > 64 ? 0.29 : s.T == 16 ? 0.27 : s.T == 32 ? 0.28 : 0.32);
+                         : (s.T > 64 ? 0.29 : s.T == 16 ? 0.27 : 0.28);
   const double w_bytes = w8 ? (double)kTileN * kTileK : (double)kTileBytes;
   constexpr double kBytesPerUs = 6.0e6;  // sustained HBM read rate
   const bool push = s.T == 16 && M <= GemmCfg<16, 9, 4, 2, true>::kPushMaxM;
@@ -241,7 +242,9 @@ Schedule choose_schedule(int M, int N, int K, int sms, bool w8, long active_m_ti
     const double t_tile = t_own > t_bw ? t_own : t_bw;
     const int lg = eff > 4 ? 3 : eff > 2 ? 2 : eff > 1 ? 1 : 0;
     const double tok = M < s.T ? M : s.T;
-    const double red = lg * (0.1 + (push ? 0.05 : 0.005 * tok));
+    // push: one async add per element into the leader, no barrier;
+    // gather: two cluster barriers and remote reads across all splits
+    const double red = eff == 1 ? 0.0 : push ? 0.1 * lg : 0.2 * eff + 0.05 * tok * lg / 8.0;
     double cost = waves * (fill + per * t_tile) + red;
     const int want = force_splits > 0 ? force_splits : forced;
     if (want > 0) cost = (eff == want) ? 0.0 : 1e6 + cost;
