@@ -27,6 +27,7 @@ __all__ = [
     "w8a8_quantize_weights", "w8a8_gemm", "w8a8_gemm_i32", "w8a8_gemm_schedule",
     "GroupedPackedWeights", "w4a8_quantize_grouped_weights", "w4a8_grouped_gemm",
     "w4a8_grouped_gemm_i32", "w4a8_grouped_gemm_schedule", "w4a8_gemm_variant", "VARIANTS",
+    "w4a8_gemm_fused", "w4a8_gemm_fused_supported",
 ]
 
 OK = 0
@@ -89,6 +90,8 @@ def lib():
             "w4a8_grouped_gemm_i32": ([p, p, i32, p, i32, i32, i32, i32, p, p], i32),
             "w4a8_grouped_gemm_schedule": ([i32, i32, i32, i32, i32, p, p, p], i32),
             "w4a8_gemm_variant": ([i32, p, p, p, i32, i32, i32, p, p, _ct.c_uint, p], i32),
+            "w4a8_gemm_fused": ([p, p, i32, i32, i32, p, _ct.c_uint, p], i32),
+            "w4a8_gemm_fused_supported": ([i32, i32, i32], i32),
             "w4a8_get_status": ([p], i32),
             "w4a8_debug_timeout_probe": ([ll, p], i32),
         }
@@ -376,6 +379,26 @@ def w4a8_gemm_variant(variant, Xq, s_x, packed, i32=False, out=None, stream=None
     rc = lib().w4a8_gemm_variant(v, _ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
                                  None, int(flags), _stream(stream))
     _check(rc, "w4a8_gemm_variant")
+    return Y
+
+
+def w4a8_gemm_fused_supported(M, N, K):
+    """Whether w4a8_gemm_fused applies to a shape (decode tiles)."""
+    return bool(lib().w4a8_gemm_fused_supported(int(M), int(N), int(K)))
+
+
+def w4a8_gemm_fused(X, packed, out=None, stream=None, flags=0):
+    """Activation quantization and the W4A8 GEMM in one launch (decode
+    shapes, see w4a8_gemm_fused_supported): Y [M, N] bf16 from fp32 X [M, K];
+    bit-identical to w4a8_quantize_act followed by w4a8_gemm."""
+    _need(X, _torch.float32, 2, "X")
+    M, K = X.shape
+    if K != packed.K:
+        raise ValueError("X has K=%d, weights have K=%d" % (K, packed.K))
+    Y = out if out is not None else _torch.empty(M, packed.N, dtype=_torch.bfloat16,
+                                                 device=X.device)
+    _check(lib().w4a8_gemm_fused(_ptr(X), _ptr(packed.data), M, packed.N, K, _ptr(Y),
+                                 int(flags), _stream(stream)), "w4a8_gemm_fused")
     return Y
 
 

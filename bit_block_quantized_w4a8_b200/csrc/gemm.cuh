@@ -51,6 +51,7 @@
 #include <cstdint>
 #include "layout.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace w4a8 {
 
@@ -96,8 +97,11 @@ struct GemmParams {
 static_assert(sizeof(GemmParams) <= 128, "kernel parameter block");
 
 template <int T, int SS, int AS, int DQG, bool PUSH = false, bool W8 = false,
-          bool PAIR = false>
+          bool PAIR = false, bool FUSED = false>
 struct GemmCfg {
+  // FUSED: the per-token activation quantization runs inside the GEMM (the
+  // 16-token light ring, every k tile of a CTA resident at once)
+  static_assert(!FUSED || (T == 16 && !W8 && !PAIR), "fused quantization: 16-token tiles");
   static_assert(T % 16 == 0 && T >= 16 && T <= 256, "MMA N for M=128");
   // PAIR: a 2-CTA cluster computes 256 channels x T tokens with CTA-pair
   // MMAs; each CTA holds its 128 channels (A and D in its tensor memory) and
@@ -128,7 +132,7 @@ struct GemmCfg {
                 "128-byte-swizzled operand tiles start on 1024-byte boundaries");
   // stage barriers: weights landed, activations landed (not in the CTA-pair
   // form, which lands both on one), stage free; slot barriers; 3 more
-  static constexpr int kNumBars = (PAIR ? 2 : 3) * SS + 2 * AS + 3;
+  static constexpr int kNumBars = (PAIR ? 2 : 3) * SS + 2 * AS + 3 + (FUSED ? 1 : 0);
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffSx = kOffMisc + 16;
   // partial tiles of at most kPushMaxM tokens are pushed (remote atomic
@@ -139,7 +143,12 @@ struct GemmCfg {
   static_assert(!PUSH || T == 16, "push reduction is for the 16-token tile");
   static constexpr int kOffRed = (kOffSx + 4 * T + 15) & ~15;
   static constexpr int kRedBytes = kPush ? T * kTileN * 4 : 0;
-  static constexpr int kSmemBytes = kOffRed + kRedBytes + 1024;  // + alignment slack
+  // fused: the cluster-wide per-token absmax (fp32 bit patterns), then this
+  // CTA's partial; the quantizing warps hold at most kFusedV float4 each
+  static constexpr int kOffAmax = kOffRed + kRedBytes;
+  static constexpr int kAmaxBytes = FUSED ? 2 * 4 * T : 0;
+  static constexpr int kFusedV = 8;
+  static constexpr int kSmemBytes = kOffAmax + kAmaxBytes + 1024;  // + alignment slack
   // the split-K partial tile reuses the pipeline buffers
   static_assert(T * kTileN * 4 <= kOffBar, "partial tile must fit the stage buffers");
 };
@@ -219,12 +228,12 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
 }
 
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8, int V, bool PAIR,
-          bool RTN>
-__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThreads, MINB)
+          bool RTN, bool FUSED>
+__global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>::kThreads, MINB)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_w,  // W8 only
                      const GemmParams p) {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>;
   // tokens per tile (MMA N): p.tn in the runtime-width instantiations,
   // else the compile-time T (which keeps the full-tile code as tight as it
   // was; a runtime width measured up to 20% slower on full tiles)
@@ -252,6 +261,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
   const uint32_t bar_acc = bar_afree + 8 * AS;
   const uint32_t bar_done = bar_acc + 8;  // every epilogue warp finished with TMEM
   const uint32_t bar_red = bar_done + 8;  // pushed partials landed (cluster leader)
+  const uint32_t bar_amax = bar_red + 8;  // fused: every split's token absmax landed
   const bool push = C::kPush && p.splits > 1 && p.M <= C::kPushMaxM;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -334,6 +344,12 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
                                                   p.group_bytes * g);
   }
 
+  // the host never launches these; stay safe anyway
+  if (FUSED && (nk > SS || t_valid * nk * (kTileK / 4) > 64 * C::kFusedV)) {
+    if (threadIdx.x == 0) record_status(kDevTimeout);
+    return;
+  }
+
   // Every warp reaches a CTA-wide barrier converged: an aligned barrier
   // reached by a warp in pieces (one lane late) can complete early and
   // leave a phase open that a later barrier then completes without waiting.
@@ -341,7 +357,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     if (lane == 0) {
       for (int s = 0; s < SS; ++s) {
         mbar_init(bar_full + 8 * s, 1);
-        if (kSplitLand) mbar_init(bar_fullx + 8 * s, 1);
+        // fused: the two quantizing warps arrive instead of a TMA
+        if (kSplitLand) mbar_init(bar_fullx + 8 * s, FUSED ? 2 : 1);
         mbar_init(bar_empty + 8 * s, 1);
       }
       for (int a = 0; a < AS; ++a) {
@@ -358,6 +375,14 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       // other split's partial (t_valid x 128 INT32 adds) has landed
       if (push && split == 0)
         mbar_arrive_expect_tx(bar_red, (uint32_t)(p.splits - 1) * (uint32_t)t_valid * kTileN * 4u);
+      if (FUSED) {
+        // split-K: every split (this CTA included) sends one max per token;
+        // one split: the quantizing warps arrive once the table is written
+        mbar_init(bar_amax, 1);
+        fence_barrier_init();
+        if (p.splits > 1)
+          mbar_arrive_expect_tx(bar_amax, (uint32_t)p.splits * (uint32_t)t_valid * 4u);
+      }
       pdl_launch_dependents();
     }
     __syncwarp();
@@ -374,6 +399,10 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     int4* red = reinterpret_cast<int4*>(smem + C::kOffRed);
     for (int i = threadIdx.x; i < C::kRedBytes / 16; i += C::kThreads)
       red[i] = make_int4(0, 0, 0, 0);
+  }
+  if (FUSED) {  // the absmax table starts at zero
+    uint32_t* tab = reinterpret_cast<uint32_t*>(smem + C::kOffAmax);
+    for (int i = threadIdx.x; i < 2 * T; i += C::kThreads) tab[i] = 0u;
   }
   tc_fence_before();
   __syncthreads();
@@ -396,6 +425,87 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     __syncthreads();
   }
 
+  // -------------------------------------- fused activation quantization
+  // Warps 0 and 1 (idle until the MMAs can start) quantize this CTA's k
+  // range of the fp32 activations straight into the stages' token tiles:
+  // the per-token absmax over the CTA's range is combined across the
+  // split-K cluster by an asynchronous max into every CTA's table, then
+  // s_x = absmax / 127 and codes rint(x / s_x) clamped to +-127 -- the rule
+  // and the arithmetic of act_quant_kernel, so the codes are the same.  The
+  // tiles are written in the 128-byte-swizzled layout the TMA would have
+  // produced (16-byte chunk c of token row t at chunk c ^ (t mod 8)).
+  auto fused_quant = [&]() {
+    const int at = warp * 32 + lane;           // 0 .. 63
+    const float* X = p.s_x;                    // fused: fp32 activations [M][K]
+    const int k_lo = kt0 * kTileK;
+    // float4 of one row in this CTA's k range (a multiple of 32), and of
+    // the whole slice; element f is float4 f % n4 of row f / n4, and the 32
+    // elements a warp holds for one j belong to one row
+    const int n4 = nk * (kTileK / 4);
+    const int total4 = t_valid * n4;  // <= 64 * C::kFusedV (host-checked)
+    uint32_t* part = reinterpret_cast<uint32_t*>(smem + C::kOffAmax) + T;  // CTA absmax [T]
+    const uint32_t tab = sbase + C::kOffAmax;
+    pdl_wait();  // X is produced by the preceding kernel
+    // every load of the slice in flight at once; the values stay in
+    // registers for the quantization below
+    float4 xv[C::kFusedV];
+#pragma unroll
+    for (int j = 0; j < C::kFusedV; ++j) {
+      const int f = at + 64 * j;
+      if (f < total4) {
+        const int t = f / n4;
+        xv[j] = __ldg(reinterpret_cast<const float4*>(X + (size_t)(row_base + t) * p.K + k_lo) +
+                      (f - t * n4));
+      } else {
+        xv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < C::kFusedV; ++j) {
+      const int f0 = 64 * j + 32 * warp;  // warp-uniform
+      if (f0 < total4) {
+        const float m = warp_max(absmax4(xv[j]));
+        if (lane == 0) atomicMax(part + f0 / n4, __float_as_uint(m));
+      }
+    }
+    named_bar_sync(2, 64);
+    if (p.splits == 1) {
+      // one CTA: the partials are the row maxima; one local arrive (no
+      // cluster addressing in a launch without clusters)
+      if (at < t_valid) reinterpret_cast<uint32_t*>(smem + C::kOffAmax)[at] = part[at];
+      named_bar_sync(2, 64);
+      if (at == 0) mbar_arrive(bar_amax);  // release: the epilogue reads the table
+    } else {
+      if (push) cluster_wait();  // every CTA's table and barrier are initialised
+      if (at < t_valid) {
+        const uint32_t v = part[at];
+        for (int q = 0; q < p.splits; ++q)
+          dsmem_red_async_max_u32(dsmem_map(tab + 4u * (uint32_t)at, (uint32_t)q), v,
+                                  dsmem_map(bar_amax, (uint32_t)q));
+      }
+      // (on a timeout the abort flag is set; no barrier below waits on these warps)
+      if (!warp_wait<true>(bar_amax, 0, abort_flag, lim)) return;
+    }
+    const uint32_t* amax = reinterpret_cast<const uint32_t*>(smem + C::kOffAmax);
+#pragma unroll
+    for (int j = 0; j < C::kFusedV; ++j) {
+      const int f = at + 64 * j;
+      if (f < total4) {
+        const int t = f / n4, i = f - t * n4;
+        const float sc = __fdiv_rn(__uint_as_float(amax[t]), 127.0f);
+        // float4 i of the row: k tile i / 32, 16-byte chunk (i / 4) % 8,
+        // word i % 4 of the chunk
+        const int it = i >> 5, c = (i >> 2) & 7;
+        sts32(sbase + it * C::kXBytes + t * 128 + ((c ^ (t & 7)) << 4) + 4 * (i & 3),
+              quant4(xv[j], sc));
+      }
+    }
+    fence_proxy_async_smem();  // the tiles above, seen by the MMA (async proxy)
+    __syncwarp();
+    if (lane == 0)
+      for (int it = 0; it < nk; ++it) mbar_arrive(bar_fullx + 8 * it);
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // The whole warp runs the loop and waits; one elected lane issues the
@@ -408,7 +518,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     const uint32_t tx_w = kSplitLand ? C::kWBytes : C::kWBytes + x_bytes;
     const uint32_t tx_x = x_bytes;
     if (leader) {
-      prefetch_tensormap(&tmap_x);
+      if (!FUSED) prefetch_tensormap(&tmap_x);  // (the fused form has no tensor maps)
       if (W8 || (p.mode & kModeStoreY)) prefetch_tensormap(&tmap_w);
     }
     const uint64_t pol =
@@ -435,16 +545,19 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
         load_w(it, it);
       }
     }
-    pdl_wait();  // activations are produced by the preceding kernel
-    if (leader) {
-      for (int it = 0; it < pre; ++it) {
-        if (kSplitLand) mbar_arrive_expect_tx(bar_fullx + 8 * it, tx_x);
-        tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
-                    row_base + rank * (TN / 2), bar_fullx + 8 * it);
+    if (!FUSED) {
+      pdl_wait();  // activations are produced by the preceding kernel
+      if (leader) {
+        for (int it = 0; it < pre; ++it) {
+          if (kSplitLand) mbar_arrive_expect_tx(bar_fullx + 8 * it, tx_x);
+          tma_load_2d(sbase + it * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
+                      row_base + rank * (TN / 2), bar_fullx + 8 * it);
+        }
       }
     }
     issued = pre;
     __syncwarp();
+    if (FUSED) fused_quant();
     for (int it = pre; it < nk; ++it) {
       const int s = it % SS;
       const uint32_t ph = (it / SS) & 1;
@@ -452,9 +565,11 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
       if (leader) {
         mbar_arrive_expect_tx(bar_full + 8 * s, tx_w);
         load_w(it, s);
-        if (kSplitLand) mbar_arrive_expect_tx(bar_fullx + 8 * s, tx_x);
-        tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
-                    row_base + rank * (TN / 2), bar_fullx + 8 * s);
+        if (!FUSED) {  // (fused calls have every k tile resident: no refills)
+          if (kSplitLand) mbar_arrive_expect_tx(bar_fullx + 8 * s, tx_x);
+          tma_load_2d(sbase + s * C::kXBytes, &tmap_x, (kt0 + it) * kTileK,
+                      row_base + rank * (TN / 2), bar_fullx + 8 * s);
+        }
       }
       __syncwarp();
       issued = it + 1;
@@ -503,6 +618,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
   } else if (warp == 1 && V != kVarGroupIssuesMma) {
     // ---------------------------------------------------------- MMA issuer
     // Whole warp waits, one elected lane issues the MMAs and commits.
+    if (FUSED) fused_quant();
     const bool leader = elect_one();
     const uint32_t idesc = idesc_i8(128, TN);
     for (int it = 0; it < nk; ++it) {
@@ -623,7 +739,15 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     const int et = threadIdx.x - 64;  // epilogue thread index
     pdl_wait();  // s_x and the outputs are ordered after the preceding kernel
     if (p.Y) {
-      for (int i = et; i < T; i += nthr) sx_s[i] = i < t_valid ? p.s_x[row_base + i] : 0.0f;
+      if (FUSED) {
+        // s_x from the cluster's absmax table (p.s_x holds the fp32 input)
+        warp_wait<true>(bar_amax, 0, abort_flag, lim);
+        const uint32_t* amax = reinterpret_cast<const uint32_t*>(smem + C::kOffAmax);
+        for (int i = et; i < T; i += nthr)
+          sx_s[i] = i < t_valid ? __fdiv_rn(__uint_as_float(amax[i]), 127.0f) : 0.0f;
+      } else {
+        for (int i = et; i < T; i += nthr) sx_s[i] = i < t_valid ? p.s_x[row_base + i] : 0.0f;
+      }
     }
     warp_wait(bar_acc, 0, abort_flag, lim);
     tc_fence_after();
@@ -842,7 +966,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>::kThre
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_done);
   }
-  if (push && warp < 2) cluster_wait();  // pairs with the arrive at set-up
+  // pairs with the arrive at set-up (the fused quantizing warps waited already)
+  if (push && warp < 2 && !FUSED) cluster_wait();
   if (warp == 1) {
     warp_wait(bar_done, 0, nullptr, lim);
     if (*abort_flag) warp_wait(bar_acc, 0, nullptr, lim);

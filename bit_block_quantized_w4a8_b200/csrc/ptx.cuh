@@ -375,6 +375,10 @@ __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void sts16(uint32_t addr, unsigned short v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -416,6 +420,23 @@ __device__ __forceinline__ void dsmem_red_async_add_s32(uint32_t caddr, int32_t 
       "red.async.relaxed.cluster.shared::cluster.mbarrier::complete_tx::bytes.add.s32 "
       "[%0], %1, [%2];" ::"r"(caddr), "r"(v), "r"(cbar)
       : "memory");
+}
+
+// Asynchronous atomic max (unsigned) into another CTA's shared memory,
+// completion counted (4 bytes) on an mbarrier in that CTA.  Non-negative
+// fp32 values order like their bit patterns, so this exchanges an absmax.
+__device__ __forceinline__ void dsmem_red_async_max_u32(uint32_t caddr, uint32_t v,
+                                                        uint32_t cbar) {
+  asm volatile(
+      "red.async.relaxed.cluster.shared::cluster.mbarrier::complete_tx::bytes.max.u32 "
+      "[%0], %1, [%2];" ::"r"(caddr), "r"(v), "r"(cbar)
+      : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // Arrive on an mbarrier in another CTA of the cluster; release at cluster

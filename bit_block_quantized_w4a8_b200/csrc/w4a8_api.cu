@@ -117,13 +117,14 @@ bool make_w8_map(CUtensorMap* map, const int8_t* Wq, int N, int K) {
 
 // -------------------------------------------------- kernel attributes
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
-          int V = kVarDefault, bool PAIR = false, bool RTN = false>
+          int V = kVarDefault, bool PAIR = false, bool RTN = false, bool FUSED = false>
 cudaError_t ensure_smem_attr() {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
-    cudaError_t e = cudaFuncSetAttribute(w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN>,
+    cudaError_t e = cudaFuncSetAttribute(
+        w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN, FUSED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -311,12 +312,12 @@ struct Maps {
 };
 
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH = false, bool W8 = false,
-          int V = kVarDefault, bool PAIR = false, bool RTN = false>
+          int V = kVarDefault, bool PAIR = false, bool RTN = false, bool FUSED = false>
 cudaError_t launch_gemm(const Maps& m, const GemmParams& p, int ctas, cudaStream_t st,
                         bool pdl) {
-  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR>;
-  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN>;
-  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN>();
+  using C = GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>;
+  auto k = w4a8_gemm_kernel<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN, FUSED>;
+  const cudaError_t ea = ensure_smem_attr<T, SS, AS, DQG, MINB, PUSH, W8, V, PAIR, RTN, FUSED>();
   if (ea != cudaSuccess) return ea;
   return launch_k(k, dim3(ctas), dim3(C::kThreads), C::kSmemBytes, st, pdl,
                   PAIR ? 2 : p.splits, m.x, m.w, p);
@@ -599,6 +600,51 @@ int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* pa
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
+// Whether the fused form (activation quantization inside the GEMM) applies:
+// the 16-token light ring with every k tile of a CTA resident, and split-K
+// only with the push reduction.
+bool fused_schedule(int M, int N, int K, int sms, Schedule* out) {
+  if (M < 1 || M > 16 || N < 1 || K % kTileK != 0 || K > 65536) return false;
+  const Schedule s = choose_schedule(M, N, K, sms, false);
+  if (s.T != 16 || ctas_per_sm(16, s.kt_per, false) != 3 || s.kt_per > 6) return false;
+  if (s.splits > 1 && M > GemmCfg<16, 6, 3, 2, true>::kPushMaxM) return false;
+  // the CTA's slice of X (M rows x kt_per k tiles) sits in the two quantizing
+  // warps' registers
+  using F = GemmCfg<16, 6, 3, 2, true, false, false, true>;
+  if (M * s.kt_per * (kTileK / 4) > 64 * F::kFusedV) return false;
+  if (out) *out = s;
+  return true;
+}
+
+int gemm_fused(const float* X, const void* packed, int M, int N, int K, uint16_t* Y,
+               unsigned flags, void* stream) {
+  if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
+  if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return W4A8_OK;
+  if (!X || !packed || !Y) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 2)) return W4A8_ERR_MISALIGNED;
+  const int dev = current_device();
+  if (dev < 0) return W4A8_ERR_CUDA;
+  Schedule s;
+  if (!fused_schedule(M, N, K, num_sms(dev), &s)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  GemmParams p = make_params(s, reinterpret_cast<const float*>(X), M, N, K, Y, nullptr);
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  p.tiles = base + tiles_offset_bytes(p.n_pad);
+  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
+  p.hdr = reinterpret_cast<const PackedHeader*>(base);
+  Maps m = {};  // no activation tensor map: the kernel reads X itself
+  const bool push = s.splits > 1;
+  const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
+  cudaStream_t st = as_stream(stream);
+  const cudaError_t e =
+      push ? launch_gemm<16, 6, 3, 2, 3, true, false, kVarDefault, false, false, true>(
+                 m, p, s.ctas, st, pdl)
+           : launch_gemm<16, 6, 3, 2, 3, false, false, kVarDefault, false, false, true>(
+                 m, p, s.ctas, st, pdl);
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
 __global__ void timeout_probe_kernel(unsigned long long limit_ns) {
   __shared__ alignas(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -767,6 +813,17 @@ int w4a8_gemm_variant(int variant, const int8_t* Xq, const float* s_x, const voi
                       int N, int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
   if (Y && acc) return W4A8_ERR_INVALID_ARG;
   return gemm_variant(variant, Xq, s_x, packed, M, N, K, Y, acc, flags, stream);
+}
+
+int w4a8_gemm_fused(const float* X, const void* packed, int M, int N, int K, uint16_t* Y,
+                    unsigned flags, void* stream) {
+  return gemm_fused(X, packed, M, N, K, Y, flags, stream);
+}
+
+int w4a8_gemm_fused_supported(int M, int N, int K) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  return fused_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev), nullptr) ? 1 : 0;
 }
 
 int w8a8_quantize_weights(const float* W, int N, int K, int8_t* Wq, float* s_w, void* stream) {

@@ -166,6 +166,35 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
                        int* ctas);
 
 /*
+ * ---- Activation quantization fused into the GEMM (decode) ----
+ * The same product as w4a8_quantize_act followed by w4a8_gemm, in one
+ * launch (the per-token quantizer of supporting citation [29] moved into the
+ * GEMM's producer): the GEMM's producer and MMA warps read the fp32
+ * activations of their k range into registers, combine the per-token absmax
+ * across the split-K cluster, and quantize straight into the MMA's operand
+ * tiles.  The rule and its arithmetic are w4a8_quantize_act's (s_x =
+ * absmax / 127, codes rint(x / s_x) clamped to +-127), so Y is bit-identical
+ * to the two-call form.
+ *   X [M][K] float32 (16-byte aligned), packed as for w4a8_gemm, Y [M][N]
+ *   bf16; all device pointers.  flags: W4A8_FLAG_PDL or 0.
+ * Applies to decode shapes only (w4a8_gemm_fused_supported): M <= 16 with
+ * the 16-token tile, at most 6 k tiles per CTA, M x (k tiles per CTA) <= 16
+ * (the CTA's slice of X fits the two warps' registers), and split-K only for
+ * M <= 8.  Other shapes return W4A8_ERR_UNSUPPORTED_SHAPE before any launch.
+ * On B200 the two calls chained with W4A8_FLAG_PDL are faster (4096 x 4096,
+ * M = 1: about 6.3 us per pair against 8.6 us): the fused kernel puts the
+ * activation reads, the cluster exchange and the quantization in front of
+ * its first MMA, where the pair overlaps the quantizer with the GEMM's weight
+ * prefetch and dequantization.
+ */
+int w4a8_gemm_fused(const float* X, const void* packed, int M, int N, int K,
+                    uint16_t* Y, unsigned flags, void* stream);
+
+/* 1 if w4a8_gemm_fused applies to the shape on the current device, else 0.
+ * Host-only. */
+int w4a8_gemm_fused_supported(int M, int N, int K);
+
+/*
  * ---- Ablation variants ----
  * The review page reports an ablation of the method's parts (referee
  * significance: LQQ, ImFP and their effect on throughput).  These variants

@@ -11,6 +11,7 @@ import torch
 import bit_block_quantized_w4a8_b200 as w4
 import oracle
 from bit_block_quantized_w4a8_b200 import workloads as wl
+from boundary_inputs import boundary_rows
 from gpu_util import assert_bf16_within_1ulp, bf16_bits, require_gpu
 
 pytestmark = pytest.mark.gpu
@@ -72,6 +73,20 @@ def test_activation_quantization_bit_exact(M, K, kind):
     Xq, sx = w4.w4a8_quantize_act(X.cuda())
     assert np.array_equal(Xq.cpu().numpy(), Xq_ref)
     assert np.array_equal(sx.cpu().numpy(), sx_ref)
+
+
+def test_activation_codes_at_rounding_boundaries():
+    # entries a few ulps either side of (k + 1/2) s_x for every code k, over
+    # scales from subnormal to huge: the codes must still be the oracle's
+    X = boundary_rows(4352)
+    Xq_ref, sx_ref = oracle.quantize_act(X)
+    Xq, sx = w4.w4a8_quantize_act(torch.from_numpy(X).cuda())
+    assert np.array_equal(sx.cpu().numpy(), sx_ref)
+    got = Xq.cpu().numpy()
+    bad = np.argwhere(got != Xq_ref)
+    assert bad.size == 0, "%d codes differ, first at %s: x=%r got %d want %d" % (
+        len(bad), tuple(bad[0]), float(X[tuple(bad[0])]), int(got[tuple(bad[0])]),
+        int(Xq_ref[tuple(bad[0])]))
 
 
 def test_activation_quantization_empty():
