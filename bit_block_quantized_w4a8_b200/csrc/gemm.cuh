@@ -764,9 +764,11 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
       if (!W8 && p.splits == 1 && (p.mode & kModeStoreY)) {
         // stage the bf16 tile as [token][128 channels] in the (free) stage
         // buffers, then one thread writes it with a TMA tensor store; rows
-        // past M and channels past N are clipped by the store
+        // past M and channels past N are clipped by the store (only the
+        // 16-column groups holding valid tokens are read from TMEM, here and
+        // below: a 256-token tile at M = 128 carries 128)
         const uint32_t ystage = sbase;
-        for (int j = dg; j < T / 16; j += DQG) {
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
           uint32_t v[16];
           tmem_ld_x16(lane_base + 16 * j, v);
           tmem_wait_ld();
@@ -787,7 +789,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         }
         __syncwarp();
       } else if (p.splits == 1) {
-        for (int j = dg; j < T / 16; j += DQG) {
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
           uint32_t v[16];
           tmem_ld_x16(lane_base + 16 * j, v);
           tmem_wait_ld();
@@ -804,7 +806,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         // (the pipeline buffers are free: every copy landed and every MMA
         // that read them completed)
         int32_t* part = reinterpret_cast<int32_t*>(smem);
-        for (int j = dg; j < T / 16; j += DQG) {
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
           uint32_t v[16];
           tmem_ld_x16(lane_base + 16 * j, v);
           tmem_wait_ld();
