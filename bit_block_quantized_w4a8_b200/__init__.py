@@ -125,6 +125,19 @@ def _need(t, dtype, ndim, name):
         raise TypeError("%s must be a contiguous %dD %s tensor" % (name, ndim, dtype))
 
 
+def _out(t, dtype, shape, like, name):
+    """The caller's output buffer, checked (the kernels write every element
+    of the given shape, so a smaller buffer would be written past), or a new
+    one on ``like``'s device."""
+    if t is None:
+        return _torch.empty(*shape, dtype=dtype, device=like.device)
+    if (not isinstance(t, _torch.Tensor) or not t.is_cuda or t.device != like.device
+            or t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous()):
+        raise TypeError("%s must be a contiguous %s tensor of shape %s on %s" %
+                        (name, dtype, tuple(shape), like.device))
+    return t
+
+
 def w4a8_status_string(code):
     return lib().w4a8_status_string(int(code)).decode()
 
@@ -157,8 +170,10 @@ def w4a8_quantize_weights(W, group=64, out=None, stream=None):
         raise W4A8Error("w4a8_packed_weight_bytes", ERR_UNSUPPORTED_SHAPE)
     if out is None:
         out = _torch.empty(nbytes, dtype=_torch.uint8, device=W.device)
-    elif out.numel() < nbytes or out.dtype != _torch.uint8:
-        raise ValueError("out must be a uint8 tensor of at least %d bytes" % nbytes)
+    elif (not isinstance(out, _torch.Tensor) or not out.is_cuda or out.device != W.device
+          or out.dtype != _torch.uint8 or out.numel() < nbytes or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous uint8 CUDA tensor of at least %d bytes "
+                         "on %s" % (nbytes, W.device))
     _check(lib().w4a8_quantize_weights(_ptr(W), N, K, group, _ptr(out), _stream(stream)),
            "w4a8_quantize_weights")
     return PackedWeights(out, N, K, group)
@@ -182,9 +197,8 @@ def w4a8_quantize_act(X, out=None, scale_out=None, stream=None, flags=0):
     ``flags`` are the launch options of w4a8_quantize_act_ex (0 = plain call)."""
     _need(X, _torch.float32, 2, "X")
     M, K = X.shape
-    Xq = out if out is not None else _torch.empty(M, K, dtype=_torch.int8, device=X.device)
-    sx = scale_out if scale_out is not None else _torch.empty(M, dtype=_torch.float32,
-                                                              device=X.device)
+    Xq = _out(out, _torch.int8, (M, K), X, "out")
+    sx = _out(scale_out, _torch.float32, (M,), X, "scale_out")
     if flags:
         rc = lib().w4a8_quantize_act_ex(_ptr(X), M, K, _ptr(Xq), _ptr(sx), int(flags),
                                         _stream(stream))
@@ -203,7 +217,7 @@ def w4a8_gemm(Xq, s_x, packed, out=None, stream=None, flags=0):
     if K != packed.K:
         raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
     N = packed.N
-    Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
+    Y = _out(out, _torch.bfloat16, (M, N), Xq, "out")
     if flags:
         rc = lib().w4a8_gemm_ex(_ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
                                 int(flags), _stream(stream))
@@ -221,7 +235,7 @@ def w4a8_gemm_i32(Xq, packed, out=None, stream=None):
     if K != packed.K:
         raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
     N = packed.N
-    acc = out if out is not None else _torch.empty(M, N, dtype=_torch.int32, device=Xq.device)
+    acc = _out(out, _torch.int32, (M, N), Xq, "out")
     _check(lib().w4a8_gemm_i32(_ptr(Xq), _ptr(packed.data), M, N, K, _ptr(acc),
                                _stream(stream)), "w4a8_gemm_i32")
     return acc
@@ -281,7 +295,7 @@ def w4a8_grouped_gemm(Xq, s_x, gw, offsets, max_rows=None, out=None, stream=None
     groups + 1 entries; ``max_rows`` bounds any group's rows (default M)."""
     _need(s_x, _torch.float32, 1, "s_x")
     M, K, max_rows = _grouped_args(Xq, gw, offsets, max_rows)
-    Y = out if out is not None else _torch.empty(M, gw.N, dtype=_torch.bfloat16, device=Xq.device)
+    Y = _out(out, _torch.bfloat16, (M, gw.N), Xq, "out")
     _check(lib().w4a8_grouped_gemm(_ptr(Xq), _ptr(s_x), _ptr(gw.data), gw.groups, _ptr(offsets),
                                    M, max_rows, gw.N, K, _ptr(Y), int(flags), _stream(stream)),
            "w4a8_grouped_gemm")
@@ -291,7 +305,7 @@ def w4a8_grouped_gemm(Xq, s_x, gw, offsets, max_rows=None, out=None, stream=None
 def w4a8_grouped_gemm_i32(Xq, gw, offsets, max_rows=None, out=None, stream=None):
     """Exact INT32 accumulators of the grouped W4A8 GEMM."""
     M, K, max_rows = _grouped_args(Xq, gw, offsets, max_rows)
-    acc = out if out is not None else _torch.empty(M, gw.N, dtype=_torch.int32, device=Xq.device)
+    acc = _out(out, _torch.int32, (M, gw.N), Xq, "out")
     _check(lib().w4a8_grouped_gemm_i32(_ptr(Xq), _ptr(gw.data), gw.groups, _ptr(offsets), M,
                                        max_rows, gw.N, K, _ptr(acc), _stream(stream)),
            "w4a8_grouped_gemm_i32")
@@ -330,7 +344,7 @@ def w8a8_gemm(Xq, s_x, Wq, s_w, out=None, stream=None, flags=0):
     if Wq.shape[1] != K or s_w.numel() != N or s_x.numel() != M:
         raise ValueError("shape mismatch: Xq %s, Wq %s, s_x %s, s_w %s"
                          % (tuple(Xq.shape), tuple(Wq.shape), s_x.numel(), s_w.numel()))
-    Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
+    Y = _out(out, _torch.bfloat16, (M, N), Xq, "out")
     _check(lib().w8a8_gemm(_ptr(Xq), _ptr(s_x), _ptr(Wq), _ptr(s_w), M, N, K, _ptr(Y),
                            int(flags), _stream(stream)), "w8a8_gemm")
     return Y
@@ -344,7 +358,7 @@ def w8a8_gemm_i32(Xq, Wq, out=None, stream=None):
     N = Wq.shape[0]
     if Wq.shape[1] != K:
         raise ValueError("Xq has K=%d, Wq has K=%d" % (K, Wq.shape[1]))
-    acc = out if out is not None else _torch.empty(M, N, dtype=_torch.int32, device=Xq.device)
+    acc = _out(out, _torch.int32, (M, N), Xq, "out")
     _check(lib().w8a8_gemm_i32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _stream(stream)),
            "w8a8_gemm_i32")
     return acc
@@ -369,13 +383,13 @@ def w4a8_gemm_variant(variant, Xq, s_x, packed, i32=False, out=None, stream=None
         raise ValueError("Xq has K=%d, weights have K=%d" % (K, packed.K))
     N = packed.N
     if i32:
-        acc = out if out is not None else _torch.empty(M, N, dtype=_torch.int32, device=Xq.device)
+        acc = _out(out, _torch.int32, (M, N), Xq, "out")
         rc = lib().w4a8_gemm_variant(v, _ptr(Xq), None, _ptr(packed.data), M, N, K, None,
                                      _ptr(acc), int(flags), _stream(stream))
         _check(rc, "w4a8_gemm_variant")
         return acc
     _need(s_x, _torch.float32, 1, "s_x")
-    Y = out if out is not None else _torch.empty(M, N, dtype=_torch.bfloat16, device=Xq.device)
+    Y = _out(out, _torch.bfloat16, (M, N), Xq, "out")
     rc = lib().w4a8_gemm_variant(v, _ptr(Xq), _ptr(s_x), _ptr(packed.data), M, N, K, _ptr(Y),
                                  None, int(flags), _stream(stream))
     _check(rc, "w4a8_gemm_variant")
@@ -395,8 +409,7 @@ def w4a8_gemm_fused(X, packed, out=None, stream=None, flags=0):
     M, K = X.shape
     if K != packed.K:
         raise ValueError("X has K=%d, weights have K=%d" % (K, packed.K))
-    Y = out if out is not None else _torch.empty(M, packed.N, dtype=_torch.bfloat16,
-                                                 device=X.device)
+    Y = _out(out, _torch.bfloat16, (M, packed.N), X, "out")
     _check(lib().w4a8_gemm_fused(_ptr(X), _ptr(packed.data), M, packed.N, K, _ptr(Y),
                                  int(flags), _stream(stream)), "w4a8_gemm_fused")
     return Y

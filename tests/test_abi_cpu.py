@@ -118,3 +118,15 @@ def test_w8a8_schedule_covers_the_machine(L):
             per = -(-kt // splits)
             assert -(-kt // per) == splits
             assert ctas == -(-N // 128) * -(-M // T) * splits
+
+
+def test_output_buffers_are_checked_before_any_launch():
+    import torch
+    like = torch.empty(2, 8)
+    assert w4._out(None, torch.int8, (2, 8), like, "out").shape == (2, 8)
+    # the kernels write every element of the output's shape: a buffer of any
+    # other shape, dtype or layout, or off the inputs' device, is refused
+    for bad in (torch.empty(2, 7, dtype=torch.int8), torch.empty(8, 2, dtype=torch.int8).t(),
+                torch.empty(2, 8, dtype=torch.int16), torch.empty(2, 8, dtype=torch.int8), "x"):
+        with pytest.raises(TypeError):
+            w4._out(bad, torch.int8, (2, 8), like, "out")

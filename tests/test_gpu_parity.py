@@ -89,6 +89,25 @@ def test_activation_codes_at_rounding_boundaries():
         int(Xq_ref[tuple(bad[0])]))
 
 
+def test_wrong_output_buffers_are_refused():
+    X = torch.randn(4, 256, device="cuda")
+    pk = w4.w4a8_quantize_weights(torch.randn(300, 256, device="cuda") * 0.02)
+    Xq, sx = w4.w4a8_quantize_act(X)
+    for bad in (torch.empty(4, 299, dtype=torch.bfloat16, device="cuda"),
+                torch.empty(4, 300, dtype=torch.float32, device="cuda"),
+                torch.empty(300, 4, dtype=torch.bfloat16, device="cuda").t()):
+        with pytest.raises(TypeError):
+            w4.w4a8_gemm(Xq, sx, pk, out=bad)
+    with pytest.raises(TypeError):
+        w4.w4a8_quantize_act(X, out=torch.empty(4, 255, dtype=torch.int8, device="cuda"))
+    with pytest.raises(TypeError):
+        w4.w4a8_quantize_act(X, scale_out=torch.empty(3, device="cuda"))
+    Y = torch.empty(4, 300, dtype=torch.bfloat16, device="cuda")
+    assert w4.w4a8_gemm(Xq, sx, pk, out=Y) is Y
+    torch.cuda.synchronize()
+    assert w4.w4a8_get_status() == 0
+
+
 def test_activation_quantization_empty():
     Xq, sx = w4.w4a8_quantize_act(torch.zeros(0, 128, device="cuda"))
     assert Xq.shape == (0, 128) and sx.shape == (0,)
