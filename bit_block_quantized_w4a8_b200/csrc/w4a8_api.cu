@@ -481,11 +481,11 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
                  : launch_gemm<16, 10, 4, 2, 2>(m, p, s.ctas, st, pdl);
       break;
     }
-    // (the 32- and 64-token tiles fill their 256 TMEM columns with A slots:
-    // more weight tiles dequantized before the activations land; 1-6% faster
-    // at M = 32..64.  The 16-token deep ring keeps 4: deeper measured slower
-    // on the long k ranges of the 70B-like decode layers)
-    case 32: e = launch_gemm<32, 8, 7, 2, 2>(m, p, s.ctas, st, pdl); break;
+    // (the 64-token tile fills its 256 TMEM columns with A slots: more weight
+    // tiles dequantized before the activations land, 4-6% faster at M = 64 on
+    // short and long k ranges.  The 16- and 32-token rings keep 4: deeper
+    // measured 2-8% slower on the long k ranges of the 70B-like decode layers)
+    case 32: e = launch_gemm<32, 8, 4, 2, 2>(m, p, s.ctas, st, pdl); break;
     case 64: e = launch_gemm<64, 6, 6, 2, 2>(m, p, s.ctas, st, pdl); break;
     case 128: e = launch_gemm<128, 4, 4, 2, 2>(m, p, s.ctas, st, pdl); break;  // tuning only
     default:
