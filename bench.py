@@ -156,6 +156,28 @@ def replica_value(units_per_rank, world, elapsed_max_s):
 
 
 # ----------------------------------------------------------------- clocks
+def gpu_local_cpus(dev):
+    """The CPUs NVML reports as local to this GPU (its NUMA node), within the
+    process's current affinity, or None when that cannot be read.  Pinned
+    host buffers allocated while the process runs there sit in the GPU's
+    local memory node, so host <-> device copies need not cross sockets."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            p = torch.cuda.get_device_properties(dev)
+            bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            words = pynvml.nvmlDeviceGetCpuAffinity(h, ((os.cpu_count() or 1) + 63) // 64)
+            cpus = {64 * i + b for i, w in enumerate(words) for b in range(64) if (w >> b) & 1}
+            cpus &= os.sched_getaffinity(0)
+            return cpus or None
+        finally:
+            pynvml.nvmlShutdown()
+    except Exception:
+        return None
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -450,10 +472,21 @@ def run_cuda(args):
     for M in Ms:
         offs[M] = m_all
         m_all += M
-    hX = torch.empty(m_all, K, dtype=torch.float32).pin_memory()
-    for M in Ms:
-        hX[offs[M]:offs[M] + M].copy_(Xs[M].cpu())
-    hY = [torch.empty(m_all, N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    # the pinned buffers are allocated (and first written) on the GPU's local
+    # CPUs, then the process's affinity is restored
+    near = gpu_local_cpus(dev)
+    saved_cpus = os.sched_getaffinity(0)
+    if near:
+        os.sched_setaffinity(0, near)
+    try:
+        hX = torch.empty(m_all, K, dtype=torch.float32).pin_memory()
+        for M in Ms:
+            hX[offs[M]:offs[M] + M].copy_(Xs[M].cpu())
+        hY = [torch.empty(m_all, N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        for t in hY:
+            t.zero_()
+    finally:
+        os.sched_setaffinity(0, saved_cpus)
     dX = [torch.empty(m_all, K, dtype=torch.float32, device=dev) for _ in range(2)]
     dY = [torch.empty(m_all, N, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -547,7 +580,9 @@ def run_cuda(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "pipeline": "one upload and one download per step on their own streams, "
                             "double-buffered against the compute stream; the step's public "
-                            "calls replayed from CUDA graphs"},
+                            "calls replayed from CUDA graphs",
+                "host_buffers": ("pinned, allocated on the GPU's local CPUs (%d)" % len(near))
+                                if near else "pinned, default placement"},
         "clocks": clk,
         "cpu_baseline": cpu,
     }
