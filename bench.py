@@ -366,6 +366,9 @@ def run_cuda(args):
     Ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in Ms}
 
     stream = torch.cuda.Stream(device=dev)
+    # the weights were packed and copied on the default stream; the timed
+    # calls run on another (non-blocking) stream
+    torch.cuda.synchronize(dev)
 
     def step_fn(r):
         def fn():
@@ -639,6 +642,7 @@ def run_all_configs(args):
                 ncopy = max(1, min(32, -(-2 * l2 // pk.data.numel())))
                 copies = [pk] + [w4.PackedWeights(pk.data.clone(), N, K, GROUP)
                                  for _ in range(ncopy - 1)]
+                torch.cuda.synchronize(dev)  # packed on the default stream; timed calls on another
                 layers_done[layer.name] = copies
             copies = layers_done[layer.name]
             X = wl.layer_activations(name, layer, M).to(dev)
@@ -711,7 +715,9 @@ def run_compare(args):
 
     def copies_of(t, nbytes):
         n = max(1, min(32, -(-2 * l2 // nbytes)))
-        return [t] + [t.clone() for _ in range(n - 1)]
+        cs = [t] + [t.clone() for _ in range(n - 1)]
+        torch.cuda.synchronize(dev)  # clones on the default stream; timed calls on another
+        return cs
 
     def timed(fn_i, n_in):
         def body():
@@ -810,6 +816,7 @@ def run_moe(args):
             act_bytes = len(active) * weight_bytes(N, K)
             ncopy = max(1, min(4, -(-2 * l2 // act_bytes)))
             copies = [data] + [data.clone() for _ in range(ncopy - 1)]
+            torch.cuda.synchronize(dev)  # packed on the default stream; timed calls on another
             gws = [w4.GroupedPackedWeights(d, w.experts, N, K, GROUP) for d in copies]
             X = wl.moe_activations(name, layer, tokens)[tok].contiguous().to(dev)
             M = X.shape[0]
@@ -897,6 +904,7 @@ def run_ablation(args):
         pk = w4.w4a8_quantize_weights(wl.layer_weights(name, layer).to(dev))
         ncopy = max(1, min(32, -(-2 * l2 // pk.data.numel())))
         copies = [pk] + [w4.PackedWeights(pk.data.clone(), N, K, GROUP) for _ in range(ncopy - 1)]
+        torch.cuda.synchronize(dev)  # packed on the default stream; timed calls on another
         for M in Ms:
             X = wl.layer_activations(name, layer, M).to(dev)
             Xq, sx = w4.w4a8_quantize_act(X)
