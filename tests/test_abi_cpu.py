@@ -130,3 +130,17 @@ def test_output_buffers_are_checked_before_any_launch():
                 torch.empty(2, 8, dtype=torch.int16), torch.empty(2, 8, dtype=torch.int8), "x"):
         with pytest.raises(TypeError):
             w4._out(bad, torch.int8, (2, 8), like, "out")
+
+
+def test_fused_call_shape_rules(L):
+    # host-only: which decode shapes the one-launch quantize + GEMM accepts
+    # (up to 16 tokens, a k range per CTA that stays resident, and the CTA's
+    # slice of X within the quantizing warps' registers); everything else is
+    # refused before any launch
+    ok = [(1, 4096, 4096), (4, 4096, 4096), (4, 28672, 512), (16, 28672, 128)]
+    refused = [(0, 4096, 4096), (8, 4096, 4096), (16, 4096, 4096), (17, 256, 4096),
+               (16, 28672, 768), (1, 4096, 4000)]
+    for sh in ok:
+        assert w4.w4a8_gemm_fused_supported(*sh), sh
+    for sh in refused:
+        assert not w4.w4a8_gemm_fused_supported(*sh), sh
