@@ -33,3 +33,15 @@ def assert_bf16_within_1ulp(got_bits: np.ndarray, ref_bits: np.ndarray, what="")
     assert d.max(initial=0) <= 1, "%s: %d outputs off by more than 1 bf16 ulp, first at %s" % (
         what, bad[0].size, tuple(int(x[0]) for x in bad))
     return d
+
+
+def check_block(acc, Y, acc_ref, y_ref, what):
+    """Every element of one block: INT32 bit-exact, bf16 within 1 ulp of the
+    FP64 epilogue, exact zero where the accumulator is zero."""
+    assert acc.shape == acc_ref.shape, what
+    bad = np.nonzero(acc != acc_ref)
+    assert bad[0].size == 0, "%s: %d accumulators differ, first at %s" % (
+        what, bad[0].size, tuple(int(x[0]) for x in bad))
+    got = bf16_bits(Y)
+    assert_bf16_within_1ulp(got, y_ref, what)
+    assert not np.any((acc_ref == 0) & ((got & 0x7FFF) != 0)), what + ": nonzero output for acc 0"

@@ -10,7 +10,7 @@ import torch
 import bit_block_quantized_w4a8_b200 as w4
 import oracle
 from bit_block_quantized_w4a8_b200 import workloads as wl
-from gpu_util import assert_bf16_within_1ulp, bf16_bits, require_gpu
+from gpu_util import assert_bf16_within_1ulp, bf16_bits, check_block, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -118,8 +118,7 @@ def test_w8a8_host_side_rejections():
 @pytest.mark.parametrize("M", [1, 8, 16, 64, 256])
 def test_w8a8_decode_sweep_full_size(M):
     """N = K = 4096 (the decode sweep) in the schedule the benchmark times:
-    sampled outputs one by one, plus exact row and column sums of every
-    accumulator."""
+    every output element against the oracle's W8A8 product."""
     N = K = 4096
     layer = wl.WORKLOADS["decode_sweep_4096"].layers[0]
     W = wl.layer_weights("decode_sweep_4096", layer)
@@ -133,16 +132,5 @@ def test_w8a8_decode_sweep_full_size(M):
     Y = w4.w8a8_gemm(Xq, sx, Wq, sw, flags=w4.W4A8_FLAG_PDL)
     torch.cuda.synchronize()
     assert w4.w4a8_get_status() == 0
-    rng = np.random.default_rng(M)
-    ms = np.concatenate([[0, M - 1, M // 2], rng.integers(0, M, 200)])
-    ns = np.concatenate([[0, N - 1, 128], rng.integers(0, N, 200)])
-    acc_s, y_s = oracle.w8a8_gemm_sampled(Xq_ref, sx_ref, Wq_ref, sw_ref, ms, ns)
-    idx_m, idx_n = torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()
-    assert np.array_equal(acc[idx_m, idx_n].cpu().numpy(), acc_s)
-    assert_bf16_within_1ulp(bf16_bits(Y[idx_m, idx_n]), y_s, "W8A8 sweep M=%d" % M)
-    colsum_w = Wq_ref.sum(axis=0, dtype=np.int64)
-    assert np.array_equal(acc.sum(dim=1, dtype=torch.int64).cpu().numpy(),
-                          Xq_ref.astype(np.int64) @ colsum_w)
-    colsum_x = Xq_ref.sum(axis=0, dtype=np.int64)
-    assert np.array_equal(acc.sum(dim=0, dtype=torch.int64).cpu().numpy(),
-                          Wq_ref.astype(np.int64) @ colsum_x)
+    acc_ref, y_ref = oracle.w8a8_gemm(Xq_ref, sx_ref, Wq_ref, sw_ref)
+    check_block(acc.cpu().numpy(), Y, acc_ref, y_ref, "W8A8 sweep M=%d" % M)
