@@ -54,7 +54,12 @@ N_COPIES = 32
 GROUP = 64
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-INT8_PER_BF16 = 2.0  # nominal dense INT8 / bf16 tensor throughput on B200
+INT8_PER_BF16 = 2.0  # nominal dense INT8 / bf16 tensor throughput on B200 (cross-check only)
+SPEC_HBM_GBS = 8000.0  # HBM3e specification figure, for context beside the measured copy rate
+# library INT8 GEMMs (cuBLASLt through torch._int_mm) whose best rate is the
+# measured dense INT8 tensor peak: the square prefill shape and the two
+# wide 70B-like shapes
+INT8_PEAK_SHAPES = ((8192, 8192, 8192), (2048, 28672, 8192), (8192, 28672, 8192))
 PDL = 1  # W4A8_FLAG_PDL: consecutive calls overlap their weight fetch with the previous kernel
 
 
@@ -89,6 +94,64 @@ def load_peaks():
     except (OSError, KeyError, ValueError):
         return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS,
                     bf16_sust=1400.0, source="fallback")
+
+
+def measure_int8_peak(dev, reps=10):
+    """Dense INT8 tensor-core peak measured on this GPU: the best of `reps`
+    runs of cuBLASLt's INT8 GEMM (torch._int_mm, INT32 output) on each shape
+    of INT8_PEAK_SHAPES, timed with CUDA events; the fastest shape is the
+    peak.  Returns (tops, per-shape figures)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(5)
+    best, per = 0.0, []
+    for M, N, K in INT8_PEAK_SHAPES:
+        A = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8).to(dev)
+        B = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8).to(dev)
+        for _ in range(3):
+            torch._int_mm(A, B.t())
+        torch.cuda.synchronize(dev)
+        t_best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(A, B.t())
+            e1.record()
+            e1.synchronize()
+            t_best = min(t_best, e0.elapsed_time(e1) / 1e3)
+        tops = 2.0 * M * N * K / t_best / 1e12
+        per.append({"M": M, "N": N, "K": K, "us": t_best * 1e6, "tops": tops})
+        best = max(best, tops)
+        del A, B
+    torch.cuda.empty_cache()
+    return best, per
+
+
+def int8_peak_tops(peaks):
+    """The tensor-bound denominator: the measured INT8 peak when there is
+    one, else the bf16 burst times the nominal INT8/bf16 ratio."""
+    return peaks.get("int8") or peaks["bf16"] * INT8_PER_BF16
+
+
+def bound_and_frac(M, N, K, seconds, peaks):
+    """Roofline of one GEMM: whichever of HBM bytes and INT8 operations takes
+    longer at peak, and the fraction of that time the GEMM achieved."""
+    hbm_t = gemm_bytes(M, N, K) / (peaks["hbm"] * 1e9)
+    tc_t = gemm_ops(M, N, K) / (int8_peak_tops(peaks) * 1e12)
+    bound = "hbm" if hbm_t >= tc_t else "tensor"
+    return bound, (hbm_t if bound == "hbm" else tc_t) / seconds
+
+
+def bench_config():
+    """The workload description shared by both arms' JSON lines."""
+    layer = wl.WORKLOADS[WORKLOAD].layers[0]
+    N, K = layer.N, layer.K
+    return {"workload": WORKLOAD, "N": N, "K": K, "Ms": list(wl.WORKLOADS[WORKLOAD].Ms),
+            "group": GROUP,
+            "step": "per M: activation quantization + W4A8 GEMM (bf16 epilogue)",
+            "l2": "inputs larger than L2: %d rotating packed weight copies (%.0f MB)"
+                  % (N_COPIES, N_COPIES * weight_bytes(N, K) / 1e6),
+            "launch": "one CUDA graph per step, programmatic dependent launch",
+            "parallelism": "replicas"}
 
 
 def csrc_digest():
@@ -273,40 +336,46 @@ def cpu_baseline(N, K, Ms, budget_s=12.0):
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step is one M=1 decode call on a
-    slice of the layer's output channels, the slice sized so that warm-up and
-    timed steps together stay within about two and a half minutes."""
+    """The oracle as the reference arm, on the sample the CUDA arm's
+    cpu_baseline times: each step is one pass over the sweep's nine M values
+    (activation quantization, dequantization, integer GEMM, FP64 epilogue per
+    M).  When warm-up and timed steps of whole passes would take longer than
+    about two and a half minutes, each pass covers the first n_sub output
+    channels of the layer instead (n_sub a multiple of 128)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     import oracle
     layer = wl.WORKLOADS[WORKLOAD].layers[0]
     N, K = layer.N, layer.K
-    wq, xs = _oracle_inputs([1])
+    Ms = list(wl.WORKLOADS[WORKLOAD].Ms)
+    wq, xs = _oracle_inputs(Ms)
+
+    def one_pass(w):
+        for M in Ms:
+            _oracle_call(xs[M], w)
     t0 = time.perf_counter()
-    _oracle_call(xs[1], wq)
+    one_pass(wq)
     t_full = time.perf_counter() - t0
     per_step = 150.0 / (args.steps + args.warmup)
-    n_sub = int(N * per_step / max(t_full, 1e-9)) // 128 * 128
-    n_sub = max(128, min(N, n_sub))
-    ws = _rows(wq, n_sub)
+    n_sub = N if t_full <= per_step else max(128, int(N * per_step / t_full) // 128 * 128)
+    ws = wq if n_sub == N else _rows(wq, n_sub)
     for _ in range(args.warmup):
-        _oracle_call(xs[1], ws)
+        one_pass(ws)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_call(xs[1], ws)
+        one_pass(ws)
     t = (time.perf_counter() - t0) / args.steps
-    value = weight_bytes(n_sub, K) / t / 1e9
-    sample = ("per step: one M=1 call on output channels [0, %d) of the N=K=%d layer "
-              "(activation quantization, dequantization, integer GEMM, FP64 epilogue)"
-              % (n_sub, K))
+    value = len(Ms) * weight_bytes(n_sub, K) / t / 1e9
+    sample = ("per step: one pass over M in %s on output channels [0, %d) of the N=K=%d layer, "
+              "each an oracle call (activation quantization, dequantization, integer GEMM, "
+              "FP64 epilogue)" % (Ms, n_sub, K))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "N": N, "K": K, "Ms": list(wl.WORKLOADS[WORKLOAD].Ms),
-                   "note": "CPU oracle on a bounded sample of the workload"},
+        "config": bench_config(),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -343,6 +412,7 @@ def run_cuda(args):
     dev = torch.device("cuda", local)
     dist_init(world, "nccl")
     peaks = load_peaks()
+    peaks["int8"], peaks["int8_shapes"] = measure_int8_peak(dev)
     layer = wl.WORKLOADS[WORKLOAD].layers[0]
     N, K = layer.N, layer.K
     Ms = list(wl.WORKLOADS[WORKLOAD].Ms)
@@ -438,9 +508,7 @@ def run_cuda(args):
         tq = _time_graph(gq, reps, stream) / N_COPIES
         t_nopdl = _time_graph(g0, reps, stream) / N_COPIES
         b, o = gemm_bytes(M, N, K), gemm_ops(M, N, K)
-        hbm_t, tc_t = b / (peaks["hbm"] * 1e9), o / (peaks["bf16"] * INT8_PER_BF16 * 1e12)
-        bound = "hbm" if hbm_t >= tc_t else "tensor"
-        frac = (hbm_t if bound == "hbm" else tc_t) / tg
+        bound, frac = bound_and_frac(M, N, K, tg, peaks)
         T, splits, ctas = w4.w4a8_gemm_schedule(M, N, K)
         per_m.append({"M": M, "gemm_us": tg * 1e6, "gemm_us_without_pdl": t_nopdl * 1e6,
                       "act_quant_us": tq * 1e6,
@@ -460,6 +528,7 @@ def run_cuda(args):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": traffic,
                 "kernel": "w4a8_gemm_kernel", "peak_source": peaks["source"],
+                "frac_of_spec": achieved / SPEC_HBM_GBS, "spec_gbs": SPEC_HBM_GBS,
                 "note": "algorithmic bytes of the nine sweep launches / their summed average "
                         "launch durations"}
 
@@ -563,17 +632,32 @@ def run_cuda(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(N, K, Ms, budget_s=args.cpu_budget)
 
+    # ---- every workload's cases (kernel timings, clocks sampled throughout);
+    # one GPU only, outside the timed region
+    all_cfg = None
+    if world == 1 and not args.no_all_configs:
+        del graphs[:], e2e_graphs[:]
+        copies.clear()
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        ck = ClockSampler(local)
+        ck.start()
+        cases = time_all_cases(w4, dev, stream, peaks)
+        all_cfg = {"clocks": ck.stop(), "targets": target_summary(cases),
+                   "timing": "each case a CUDA graph of back-to-back launches with programmatic "
+                             "dependent launch over rotating weight copies larger than twice the "
+                             "L2; CUDA events on the launching stream",
+                   "cases": [{k: c[k] for k in ("workload", "layer", "M", "N", "K", "gemm_us",
+                                                "tops", "weight_gbs", "bound", "frac",
+                                                "act_quant_us", "status", "schedule")}
+                             for c in cases]}
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": elapsed_max / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "N": N, "K": K, "Ms": Ms, "group": GROUP,
-                   "step": "per M: activation quantization + W4A8 GEMM (bf16 epilogue)",
-                   "l2": "inputs larger than L2: %d rotating packed weight copies (%.0f MB)"
-                         % (N_COPIES, N_COPIES * w4.w4a8_packed_weight_bytes(N, K) / 1e6),
-                   "launch": "one CUDA graph per step, programmatic dependent launch",
-                   "parallelism": "replicas"},
+        "config": bench_config(),
         "tops": tops,
         "gpu_launches": 2 * len(Ms) * args.steps,
         "roofline": roofline,
@@ -588,10 +672,19 @@ def run_cuda(args):
                                 if near else "pinned, default placement"},
         "clocks": clk,
         "cpu_baseline": cpu,
+        "peaks": {"hbm_gbs": peaks["hbm"], "hbm_source": peaks["source"],
+                  "int8_tops": peaks["int8"],
+                  "int8_source": "measured: best cuBLASLt INT8 GEMM (torch._int_mm) of %s"
+                                 % ["%dx%dx%d" % (d["M"], d["N"], d["K"])
+                                    for d in peaks["int8_shapes"]],
+                  "int8_shapes": peaks["int8_shapes"],
+                  "int8_nominal_from_bf16": peaks["bf16"] * INT8_PER_BF16},
+        "all_configs": all_cfg,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     graphs.clear()
+    e2e_graphs.clear()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -616,19 +709,14 @@ def run_profile_case(args):
     return 0 if status == 0 else 1
 
 
-def run_all_configs(args):
+def time_all_cases(w4, dev, stream, peaks, verbose=True):
     """Kernel timings on every synthetic workload (all layers and M values):
     per case the GEMM and the activation quantizer are each timed as graphs
     of back-to-back launches (programmatic dependent launch), with enough
     rotating weight copies that the working set exceeds twice the L2.
-    Writes one JSON document to ``args.all_configs``."""
-    import bit_block_quantized_w4a8_b200 as w4
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
-    peaks = load_peaks()
+    Returns one dict per case."""
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    stream = torch.cuda.Stream(device=dev)
-    out = {"peaks": peaks, "cases": []}
+    cases = []
     for name in wl.WORKLOADS:
         layers_done = {}
         for M, layer in wl.cases(name):
@@ -672,22 +760,56 @@ def run_all_configs(args):
             tq = _time_graph(gq, reps, stream) / reps_in
             status = w4.w4a8_get_status(stream)
             b, o = gemm_bytes(M, N, K), gemm_ops(M, N, K)
-            hbm_t, tc_t = b / (peaks["hbm"] * 1e9), o / (peaks["bf16"] * INT8_PER_BF16 * 1e12)
-            bound = "hbm" if hbm_t >= tc_t else "tensor"
+            bound, frac = bound_and_frac(M, N, K, tg, peaks)
             T, splits, ctas = w4.w4a8_gemm_schedule(M, N, K)
             case = {"workload": name, "layer": layer.name, "M": M, "N": N, "K": K,
                     "gemm_us": tg * 1e6, "tops": o / tg / 1e12,
                     "weight_gbs": weight_bytes(N, K) / tg / 1e9, "total_gbs": b / tg / 1e9,
-                    "bound": bound, "frac": (hbm_t if bound == "hbm" else tc_t) / tg,
+                    "bound": bound, "frac": frac,
                     "act_quant_us": tq * 1e6, "act_quant_gbs": act_bytes(M, K) / tq / 1e9,
                     "weight_copies": len(copies), "status": status,
                     "schedule": {"tile_tokens": T, "splits": splits, "ctas": ctas}}
-            out["cases"].append(case)
-            print("%-18s %-9s M=%-6d %9.2f us %8.1f TOPS %7.0f wGB/s %-6s %.3f  (%s)" % (
-                name, layer.name, M, case["gemm_us"], case["tops"], case["weight_gbs"], bound,
-                case["frac"], case["schedule"]), flush=True)
-            del gg, gq
+            cases.append(case)
+            if verbose:
+                print("%-18s %-9s M=%-6d %9.2f us %8.1f TOPS %7.0f wGB/s %-6s %.3f  (%s)" % (
+                    name, layer.name, M, case["gemm_us"], case["tops"], case["weight_gbs"],
+                    bound, case["frac"], case["schedule"]), file=sys.stderr, flush=True)
+            del gg, gq, X, Xq, sx, Y
         layers_done.clear()
+    torch.cuda.empty_cache()
+    return cases
+
+
+def target_summary(cases):
+    """The two targets over the timed cases: HBM fraction at M <= 16 and INT8
+    tensor fraction at M >= 4096 (lowest and highest of each)."""
+    small = [c["frac"] for c in cases if c["M"] <= 16 and c["bound"] == "hbm"]
+    large = [c["frac"] for c in cases if c["M"] >= 4096 and c["bound"] == "tensor"]
+    out = {}
+    if small:
+        out["hbm_frac_at_M_le_16"] = {"min": min(small), "max": max(small), "cases": len(small),
+                                      "target": 0.70}
+    if large:
+        out["int8_frac_at_M_ge_4096"] = {"min": min(large), "max": max(large),
+                                         "cases": len(large), "target": 0.60}
+    return out
+
+
+def run_all_configs(args):
+    """--all-configs PATH: every workload case timed (``time_all_cases``),
+    the INT8 peak measured first and the clocks sampled throughout; one JSON
+    document to PATH."""
+    import bit_block_quantized_w4a8_b200 as w4
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    peaks["int8"], peaks["int8_shapes"] = measure_int8_peak(dev)
+    stream = torch.cuda.Stream(device=dev)
+    clocks = ClockSampler(0)
+    clocks.start()
+    cases = time_all_cases(w4, dev, stream, peaks)
+    out = {"peaks": peaks, "clocks": clocks.stop(), "cases": cases,
+           "targets": target_summary(cases)}
     with open(args.all_configs, "w") as f:
         json.dump(out, f, indent=1)
     return 0
@@ -705,6 +827,9 @@ def run_compare(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
+    peaks["int8"], peaks["int8_shapes"] = measure_int8_peak(dev)
+    clocks = ClockSampler(0)
+    clocks.start()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     stream = torch.cuda.Stream(device=dev)
     shapes = [("decode_sweep_4096", "square", [1, 4, 16, 64, 128, 256]),
@@ -780,6 +905,7 @@ def run_compare(args):
             print("%-18s %-6s M=%-5d " % (name, lname, M) + "  ".join(
                 "%s %.2fus" % (k, v * 1e6) for k, v in t.items()), flush=True)
         del c64, c128, c8, cbf, p64, p128, pk64, pk128, Wq, sw, Wbf
+    out["clocks"] = clocks.stop()
     with open(args.compare, "w") as f:
         json.dump(out, f, indent=1)
     return 0
@@ -796,6 +922,9 @@ def run_moe(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
+    peaks["int8"], peaks["int8_shapes"] = measure_int8_peak(dev)
+    clocks = ClockSampler(0)
+    clocks.start()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     stream = torch.cuda.Stream(device=dev)
     name = "mixtral_like"
@@ -852,7 +981,7 @@ def run_moe(args):
             status = w4.w4a8_get_status(stream)
             ops = 2.0 * M * N * K
             tot_bytes = act_bytes + M * K + 4 * M + 2 * M * N
-            hbm_t, tc_t = tot_bytes / (peaks["hbm"] * 1e9), ops / (peaks["bf16"] * INT8_PER_BF16 * 1e12)
+            hbm_t, tc_t = tot_bytes / (peaks["hbm"] * 1e9), ops / (int8_peak_tops(peaks) * 1e12)
             bound = "hbm" if hbm_t >= tc_t else "tensor"
             tg = t["grouped"]
             T, splits, ctas = w4.w4a8_grouped_gemm_schedule(w.experts, M, mr, N, K)
@@ -873,6 +1002,7 @@ def run_moe(args):
                       case["schedule"]), flush=True)
             del copies, gws
         del data
+    out["clocks"] = clocks.stop()
     with open(args.moe, "w") as f:
         json.dump(out, f, indent=1)
     return 0
@@ -888,6 +1018,9 @@ def run_ablation(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
+    peaks["int8"], peaks["int8_shapes"] = measure_int8_peak(dev)
+    clocks = ClockSampler(0)
+    clocks.start()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     stream = torch.cuda.Stream(device=dev)
     shapes = [("decode_sweep_4096", "square", [1, 16, 256]),
@@ -938,6 +1071,7 @@ def run_ablation(args):
             print("%-18s %-9s M=%-5d " % (name, lname, M) + "  ".join(
                 "%s %.2fus" % (k, x * 1e6) for k, x in t.items()), flush=True)
         del copies, pk
+    out["clocks"] = clocks.stop()
     with open(args.ablation, "w") as f:
         json.dump(out, f, indent=1)
     return 0
@@ -950,6 +1084,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-all-configs", action="store_true",
+                    help="skip the per-case timings of every workload after the timed run")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU work for the oracle baseline sample")
     ap.add_argument("--profile", default=None,

@@ -52,6 +52,8 @@ struct PackedHeader {
   uint64_t tiles_offset;
   uint64_t total_bytes;
 };
+static_assert(sizeof(PackedHeader) == 48 && sizeof(PackedHeader) <= kHeaderBytes,
+              "packed header fields");
 
 __host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 

@@ -51,6 +51,16 @@ __global__ void __launch_bounds__(256) weight_scale_kernel(
     h.total_bytes = packed_bytes(N, K);
     *reinterpret_cast<PackedHeader*>(packed) = h;
   }
+  if (blockIdx.x == 0) {
+    // the rest of the header and the gap between the scales and the first
+    // tile are zero, so every byte of the buffer is defined
+    for (uint32_t i = sizeof(PackedHeader) + threadIdx.x; i < (uint32_t)kHeaderBytes;
+         i += blockDim.x)
+      packed[i] = 0;
+    const uint64_t gap0 = sw_offset_bytes() + 4ull * (uint64_t)n_pad;
+    const uint64_t gap1 = tiles_offset_bytes(n_pad);
+    for (uint64_t i = gap0 + threadIdx.x; i < gap1; i += blockDim.x) packed[i] = 0;
+  }
   if (warp >= n_pad) return;
   float amax = 0.0f;
   if (warp < N) {

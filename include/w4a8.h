@@ -33,7 +33,12 @@
  *     K <= 65536, group = 64 or 128.  M == 0 is a no-op.  Other shapes return
  *     W4A8_ERR_UNSUPPORTED_SHAPE before anything is launched.
  *   - Alignment: Xq, X, W and the packed buffer must be 16-byte aligned,
- *     Y and acc 4-byte aligned; otherwise W4A8_ERR_MISALIGNED.
+ *     acc and every float32 scale array 4-byte aligned, Y 2-byte aligned;
+ *     otherwise W4A8_ERR_MISALIGNED.  Y only needs its element alignment;
+ *     a more aligned Y enables faster stores: 16-byte alignment with N a
+ *     multiple of 8 lets dense calls without split-K write whole tiles with
+ *     a TMA tensor store, 8-byte alignment with N a multiple of 4 lets
+ *     split-K reductions store four channels per instruction.
  *   - Return value: W4A8_OK or a negative w4a8_status.  Argument errors are
  *     detected on the host before any launch.  A launch failure returns
  *     W4A8_ERR_CUDA.  Errors found on the device (a bounded wait that ran out)
@@ -84,7 +89,8 @@ size_t w4a8_packed_weight_bytes(int N, int K, int group);
  * summary; referee major 3 and minor 2, paper Sec. 4 Eqs. 7 and 10).
  *   W       [N][K] float32, device
  *   packed  device buffer of w4a8_packed_weight_bytes(N, K, group) bytes,
- *           fully written by this call (padding included)
+ *           every byte written by this call (header tail and padding
+ *           channels included), so the buffer can be saved and reloaded
  * Level 1: s_w[n] = max_k |W[n][k]| / 119 (fp32 division);
  *          Q = clamp(rint(W / s_w), -119, 119), ties to even; s_w = 0 gives 0.
  * Level 2, per group of `group` k-values in one row: mn/mx = min/max of Q,

@@ -252,6 +252,30 @@ def test_packed_header_mismatch_is_reported():
     assert int((out != 7).sum()) == 0
 
 
+@pytest.mark.parametrize("N,K", [(256, 256), (200, 384)])
+def test_packed_buffer_every_byte_written(N, K):
+    """A buffer pre-filled with garbage comes back fully defined: the header
+    beyond its fields and the gap before the first tile are zero, padding
+    channels have zero scales, and two packings of the same weights into
+    differently pre-filled buffers are byte-identical (the buffer can be
+    saved and reloaded)."""
+    W = wl.random_matrix(N, K, 13, std=0.02).cuda()
+    nbytes = w4.w4a8_packed_weight_bytes(N, K)
+    outs = []
+    for fill in (0xAB, 0x00):
+        buf = torch.full((nbytes,), fill, dtype=torch.uint8, device="cuda")
+        w4.w4a8_quantize_weights(W, out=buf)
+        outs.append(buf.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])
+    b = outs[0]
+    n_pad = -(-N // 128) * 128
+    assert not b[48:256].any()
+    sw_end = 256 + 4 * n_pad
+    tiles = -(-sw_end // 256) * 256
+    assert not b[sw_end:tiles].any()
+    assert not b[256 + 4 * N:sw_end].any()  # scales of the padding channels
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     w4.w4a8_debug_timeout_probe(2_000_000)  # 2 ms limit, nothing ever arrives
     assert w4.w4a8_get_status() == w4.ERR_TIMEOUT
