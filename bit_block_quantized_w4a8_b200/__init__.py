@@ -27,7 +27,8 @@ __all__ = [
     "w8a8_quantize_weights", "w8a8_gemm", "w8a8_gemm_i32", "w8a8_gemm_schedule",
     "GroupedPackedWeights", "w4a8_quantize_grouped_weights", "w4a8_grouped_gemm",
     "w4a8_grouped_gemm_i32", "w4a8_grouped_gemm_schedule", "w4a8_gemm_variant", "VARIANTS",
-    "w4a8_gemm_fused", "w4a8_gemm_fused_supported",
+    "w4a8_gemm_fused", "w4a8_gemm_fused_supported", "w4a8_gemm_kernel_kind",
+    "KERNEL_TENSOR_CORE", "KERNEL_WARP_MMA", "w4a8_debug_set_wait_budget",
 ]
 
 OK = 0
@@ -40,10 +41,16 @@ ERR_BAD_PACKED = -7
 ERR_BAD_OFFSETS = -8
 
 W4A8_FLAG_PDL = 1  # programmatic dependent launch (see include/w4a8.h)
+W4A8_FLAG_TENSOR_CORE = 2  # the tcgen05 kernel even where the decode form applies
 
 # kernel variants of the ablation study (W4A8_VARIANT_* in include/w4a8.h)
 VARIANTS = {"default": 0, "baseline": 1, "naive_dequant": 2, "serial": 3, "one_group": 4,
-            "group_issues_mma": 5, "cta_pair": 6}
+            "group_issues_mma": 5, "cta_pair": 6, "tensor_core": 7, "dp4a": 8,
+            "warp_mma": 9}
+
+# kernels behind w4a8_gemm (W4A8_KERNEL_* in include/w4a8.h)
+KERNEL_TENSOR_CORE = 0
+KERNEL_WARP_MMA = 1
 
 
 class W4A8Error(RuntimeError):
@@ -82,6 +89,7 @@ def lib():
             "w4a8_gemm": ([p, p, p, i32, i32, i32, p, p], i32),
             "w4a8_gemm_i32": ([p, p, i32, i32, i32, p, p], i32),
             "w4a8_gemm_schedule": ([i32, i32, i32, p, p, p], i32),
+            "w4a8_gemm_kernel_kind": ([i32, i32, i32], i32),
             "w8a8_quantize_weights": ([p, i32, i32, p, p, p], i32),
             "w8a8_gemm": ([p, p, p, p, i32, i32, i32, p, _ct.c_uint, p], i32),
             "w8a8_gemm_i32": ([p, p, i32, i32, i32, p, p], i32),
@@ -94,6 +102,7 @@ def lib():
             "w4a8_gemm_fused_supported": ([i32, i32, i32], i32),
             "w4a8_get_status": ([p], i32),
             "w4a8_debug_timeout_probe": ([ll, p], i32),
+            "w4a8_debug_set_wait_budget": ([ll], i32),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -396,6 +405,15 @@ def w4a8_gemm_variant(variant, Xq, s_x, packed, i32=False, out=None, stream=None
     return Y
 
 
+def w4a8_gemm_kernel_kind(M, N, K):
+    """Which kernel w4a8_gemm runs for a shape: KERNEL_TENSOR_CORE or
+    KERNEL_WARP_MMA (the decode form for a few tokens)."""
+    k = lib().w4a8_gemm_kernel_kind(int(M), int(N), int(K))
+    if k < 0:
+        raise W4A8Error("w4a8_gemm_kernel_kind", k)
+    return k
+
+
 def w4a8_gemm_fused_supported(M, N, K):
     """Whether w4a8_gemm_fused applies to a shape (decode tiles)."""
     return bool(lib().w4a8_gemm_fused_supported(int(M), int(N), int(K)))
@@ -423,3 +441,9 @@ def w4a8_get_status(stream=None):
 def w4a8_debug_timeout_probe(limit_ns, stream=None):
     _check(lib().w4a8_debug_timeout_probe(int(limit_ns), _stream(stream)),
            "w4a8_debug_timeout_probe")
+
+
+def w4a8_debug_set_wait_budget(ns):
+    """Test aid: budget of the kernels' main-loop waits for later launches
+    (-1 = the default 2 s; 0 = expire at once, so every launch aborts)."""
+    _check(lib().w4a8_debug_set_wait_budget(int(ns)), "w4a8_debug_set_wait_budget")

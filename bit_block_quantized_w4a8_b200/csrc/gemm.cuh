@@ -577,8 +577,9 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
     if (*abort_flag) {
       // let the copies already issued land before the CTA goes away
       for (int it = issued - SS < 0 ? 0 : issued - SS; it < issued; ++it) {
-        mbar_wait(bar_full + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
-        if (kSplitLand) mbar_wait(bar_fullx + 8 * (it % SS), (it / SS) & 1, nullptr, lim);
+        mbar_wait(bar_full + 8 * (it % SS), (it / SS) & 1, nullptr, kDrainLimitNs);
+        if (kSplitLand)
+          mbar_wait(bar_fullx + 8 * (it % SS), (it / SS) & 1, nullptr, kDrainLimitNs);
       }
     }
     __syncwarp();  // reconverge before any CTA- or cluster-wide barrier
@@ -851,7 +852,9 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         }
         __syncwarp();
       } else {
-        warp_wait<true>(bar_red, 0, abort_flag, lim);  // remote arrivals: cluster scope
+        // remote arrivals (cluster scope); the full budget even after this
+        // CTA's own abort: the other splits' adds land in its memory
+        warp_wait<true>(bar_red, 0, nullptr, kDrainLimitNs);
         if (*ep_flag) {
           const int32_t* rb = reinterpret_cast<const int32_t*>(smem + C::kOffRed);
           for (int j = dg; j < T / 16; j += DQG) {
@@ -877,8 +880,24 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
 
   if (p.splits > 1 && !push) {
     // ---------------------- split-K by gathering partials over the cluster
-    cluster_sync_all();  // every partial of the cluster is in shared memory
-    if (warp >= 2 && *ep_flag) {
+    cluster_sync_all();  // every partial (and every split's ep_flag) is in shared memory
+    // a split that aborted wrote no partial: store nothing unless every
+    // split of the cluster completed (one remote read per split and warp)
+    bool all_ok = false;
+    if (warp >= 2) {
+      int ok = 1;
+      if (lane == 0) {
+        const uint32_t epa = sbase + C::kOffMisc + 12;
+        int got[kClusterMax];
+#pragma unroll
+        for (int q = 0; q < kClusterMax; ++q)
+          got[q] = q < p.splits ? dsmem_ld_s32(dsmem_map(epa, (uint32_t)q)) : 1;
+#pragma unroll
+        for (int q = 0; q < kClusterMax; ++q) ok &= got[q] != 0;
+      }
+      all_ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+    }
+    if (warp >= 2 && all_ok) {
       const int nthr = 128 * DQG;
       const int et = threadIdx.x - 64;
       const int total = t_valid * kTileN;
@@ -976,8 +995,13 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
   // pairs with the arrive at set-up (the fused quantizing warps waited already)
   if (push && warp < 2 && !FUSED) cluster_wait();
   if (warp == 1) {
-    warp_wait(bar_done, 0, nullptr, lim);
-    if (*abort_flag) warp_wait(bar_acc, 0, nullptr, lim);
+    // after an abort the commit on bar_acc tracks every MMA issued; each
+    // completes within microseconds, so with the full drain budget this wait
+    // ends with the MMAs done and tensor memory is never freed under them
+    warp_wait(bar_done, 0, nullptr, kDrainLimitNs);
+    if (*abort_flag) warp_wait(bar_acc, 0, nullptr, kDrainLimitNs);
+    // fused split-K: every split's absmax (sent unconditionally) has landed
+    if (FUSED && p.splits > 1) warp_wait<true>(bar_amax, 0, nullptr, kDrainLimitNs);
     tc_fence_after();
     if (PAIR)
       tmem_dealloc_pair(tmem, C::kTmemCols);

@@ -18,6 +18,12 @@ __device__ __forceinline__ void record_status(int code) {
   atomicCAS(&g_status, 0, code);
 }
 
+// Budget of the waits that drain work already in flight after an abort
+// (copies issued, MMAs issued, remote adds on their way): always the full
+// 2 s, whatever the main loop's budget, so a CTA never frees tensor memory
+// or exits while an asynchronous operation can still write to it.
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -96,10 +102,17 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // after `limit_ns` of global time or as soon as *abort is set by another
 // role of the CTA; on giving up it records kDevTimeout (once per device),
 // raises *abort so the other roles leave their loops too, and returns false.
+// A budget of 0 (a test aid, never used by the library's own calls) makes
+// the wait expire at once, so the abort path runs deterministically.
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int* abort,
                                           uint64_t limit_ns) {
+  if (limit_ns == 0) {
+    record_status(kDevTimeout);
+    if (abort) *abort = 1;
+    return false;
+  }
   auto test = [&]() {
     return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
   };
@@ -137,6 +150,38 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::"
       "bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// 3-D and 4-D tiled tensor copies global -> shared: the box at the given
+// coordinates lands in shared memory innermost dimension first; elements
+// outside the tensor are zero-filled and still counted in the byte total.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::"
+      "bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, int w, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::"
+      "bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
+
+// 1-D bulk copy global -> shared without a cache hint.  dst, src 16-byte
+// aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s_plain(uint32_t dst, const void* src, uint32_t bytes,
+                                               uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
 

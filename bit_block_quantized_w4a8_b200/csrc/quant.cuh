@@ -8,9 +8,12 @@
 // (referee summary; referee minor 2, Sec. 4 Eq. 10); offset a = 2^7 + min
 // (key_machinery); per-token INT8 activations (supporting citation [29]).
 //
-// Every FP -> integer decision uses IEEE fp32 division (__fdiv_rn, never a
-// reciprocal) and round-half-to-even (__float2int_rn), so codes are exactly
-// reproducible on any IEEE machine.
+// Every FP -> integer decision rounds the correctly rounded fp32 quotient
+// x / s half-to-even (__float2int_rn): the IEEE division __fdiv_rn, or for
+// activation rows with a scale in [2^-90, 2^90] the same quotient reached
+// through the correctly rounded reciprocal and one exact-residual
+// correction (quant_sym_rcp).  Codes are therefore exactly reproducible on
+// any IEEE machine.
 #pragma once
 #include <cstdint>
 #include "layout.cuh"
@@ -202,6 +205,33 @@ __device__ __forceinline__ uint32_t quant4(float4 v, float s) {
          ((uint32_t)(quant_sym(v.w, s, 127) & 0xFF) << 24);
 }
 
+// The same codes without a division per element: with y = RN(1/s) (one
+// IEEE division per row), q = RN(x * y), the residual r = x - q * s computed
+// exactly by one fused multiply-add, and q' = RN(q + r * y), q' is the
+// correctly rounded quotient RN(x / s) (Markstein's theorem on division by
+// a correctly rounded reciprocal with one correction step; it needs the
+// residual exact and normal, which holds for 2^-90 <= s <= 2^90 and
+// |x| <= 127.5 s).  So rint(q') is exactly the code of quant_sym.  Rows
+// whose scale is outside that range (or zero) take quant4 instead.
+__device__ __forceinline__ bool rcp_quant_ok(float s) {
+  return s >= 0x1p-90f && s <= 0x1p90f;
+}
+
+__device__ __forceinline__ int quant_sym_rcp(float x, float s, float y, int range) {
+  float q = __fmul_rn(x, y);
+  const float r = __fmaf_rn(-q, s, x);
+  q = __fmaf_rn(r, y, q);
+  const int c = __float2int_rn(q);
+  return c > range ? range : (c < -range ? -range : c);
+}
+
+__device__ __forceinline__ uint32_t quant4_rcp(float4 v, float s, float y) {
+  return (uint32_t)(quant_sym_rcp(v.x, s, y, 127) & 0xFF) |
+         ((uint32_t)(quant_sym_rcp(v.y, s, y, 127) & 0xFF) << 8) |
+         ((uint32_t)(quant_sym_rcp(v.z, s, y, 127) & 0xFF) << 16) |
+         ((uint32_t)(quant_sym_rcp(v.w, s, y, 127) & 0xFF) << 24);
+}
+
 __device__ __forceinline__ float absmax4(float4 v) {
   return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 }
@@ -237,13 +267,27 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
   const float s = __fdiv_rn(red[0], 127.0f);
   if (threadIdx.x == 0) s_x[m] = s;
   uint32_t* out = reinterpret_cast<uint32_t*>(Xq + (size_t)m * K);
+  // (the branch is uniform over the row; the per-element IEEE division of
+  // quant4 carries a slow-path branch for every element, which measured
+  // about 1.1 us for 16 values per thread on a one-row launch)
+  if (rcp_quant_ok(s)) {
+    const float y = __fdiv_rn(1.0f, s);
 #pragma unroll
-  for (int i = 0; i < kActRegs; ++i) {
-    const int idx = threadIdx.x + i * kActThreads;
-    if (idx < n4) out[idx] = quant4(v[i], s);
+    for (int i = 0; i < kActRegs; ++i) {
+      const int idx = threadIdx.x + i * kActThreads;
+      if (idx < n4) out[idx] = quant4_rcp(v[i], s, y);
+    }
+    for (int idx = threadIdx.x + kActRegs * kActThreads; idx < n4; idx += kActThreads)
+      out[idx] = quant4_rcp(__ldg(row + idx), s, y);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kActRegs; ++i) {
+      const int idx = threadIdx.x + i * kActThreads;
+      if (idx < n4) out[idx] = quant4(v[i], s);
+    }
+    for (int idx = threadIdx.x + kActRegs * kActThreads; idx < n4; idx += kActThreads)
+      out[idx] = quant4(__ldg(row + idx), s);
   }
-  for (int idx = threadIdx.x + kActRegs * kActThreads; idx < n4; idx += kActThreads)
-    out[idx] = quant4(__ldg(row + idx), s);
 }
 
 }  // namespace w4a8

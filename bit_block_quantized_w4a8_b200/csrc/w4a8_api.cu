@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "gemm.cuh"
+#include "gemv.cuh"
 #include "layout.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -27,6 +28,14 @@ namespace {
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kMaxDevices = 64;
+
+// Budget of the kernels' main-loop waits: 2 s, or a test budget set by
+// w4a8_debug_set_wait_budget (0 = every such wait expires at once).
+std::atomic<long long> g_wait_budget{-1};
+unsigned long long wait_budget() {
+  const long long v = g_wait_budget.load(std::memory_order_relaxed);
+  return v < 0 ? kWaitLimitNs : (unsigned long long)v;
+}
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -360,7 +369,7 @@ cudaError_t launch_pair(const int8_t* Xq, int M, int K, Maps& m, GemmParams& p, 
 // of the parameters.  Returns W4A8_OK or an error (nothing launched).
 int check_common(const int8_t* Xq, const float* s_x, const void* w, int M, int N, int K,
                  uint16_t* Y, int32_t* acc, unsigned flags) {
-  if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)(W4A8_FLAG_PDL | W4A8_FLAG_TENSOR_CORE)) return W4A8_ERR_INVALID_ARG;
   if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
   if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return W4A8_OK;
@@ -393,7 +402,7 @@ GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K,
   p.kt_per_split = s.kt_per;
   p.n_tiles = s.n_tiles;
   p.m_tiles = s.m_tiles;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.wait_limit_ns = wait_budget();
   p.hdr = nullptr;
   p.offsets = nullptr;
   p.group_bytes = 0;
@@ -412,6 +421,153 @@ GemmParams make_params(const Schedule& s, const float* s_x, int M, int N, int K,
   return p;
 }
 
+// ------------------------------------------------ CUDA-core decode form
+// (gemv.cuh): R = 16 channels per CTA, P = 8 pieces per thread, so a CTA
+// covers at most 32 k tiles (K = 4096); longer rows split K across a cluster.
+constexpr int kGemvR = 16, kGemvP = 8, kGemvMinB = 2;
+using GemvC = GemvCfg<kGemvR, kGemvP>;
+// the warp-MMA form covers the same CTA slice (16 channels x 32 k tiles)
+using GemvMmaC = GemvMmaCfg<GemvC::kKR>;
+static_assert(GemvMmaC::kR == kGemvR, "one tensor-map box for both decode forms");
+
+struct GemvSchedule {
+  int splits = 1, kt_per = 1, ctas = 0;
+};
+
+// Whether the CUDA-core form applies to a shape (fused: one split only, the
+// CTA then holds whole rows of X for the per-token absmax).
+bool gemv_schedule(int M, int N, int K, bool fused, GemvSchedule* out) {
+  if (M < 1 || M > kGemvMaxM || N < 1 || K < kTileK || K % kTileK != 0 || K > 65536)
+    return false;
+  const int kt = K / kTileK;
+  const int splits = (kt + GemvC::kKR - 1) / GemvC::kKR;
+  if (splits > kGemvMaxSplits || (fused && splits > 1)) return false;
+  GemvSchedule s;
+  s.splits = splits;
+  s.kt_per = (kt + splits - 1) / splits;
+  s.ctas = round_up(N, kTileN) / kGemvR * splits;
+  if (out) *out = s;
+  return true;
+}
+
+// W4A8_GEMV=0 in the environment never takes the CUDA-core form, =1 takes
+// it wherever it applies (tuning experiments only).
+int gemv_env() {
+  static const int v = [] {
+    const char* e = getenv("W4A8_GEMV");
+    return e ? (e[0] == '0' ? 0 : 1) : -1;
+  }();
+  return v;
+}
+
+// Default choice between the decode form and the tcgen05 kernel: the decode
+// form when all its CTAs are resident at once (two per SM), so that every
+// CTA fetches and dequantizes its weights before the preceding kernel
+// finishes.  Measured on B200 (graphs of back-to-back calls with
+// programmatic dependent launch): N = K = 4096, M = 1..8: 4.6-4.8 us
+// against 5.0-5.7 us, and 6.0-6.7 us against 6.3-8.5 us per quantize +
+// GEMM pair; with several waves of CTAs (7B- and 70B-like layers) each
+// wave waits for its weights and the tcgen05 kernel is 1.5-2.5x faster.
+bool prefer_gemv(int M, int N, int K) {
+  GemvSchedule s;
+  if (!gemv_schedule(M, N, K, false, &s)) return false;
+  const int env = gemv_env();
+  if (env >= 0) return env == 1;
+  int dev = 0;
+  const int sms = cudaGetDevice(&dev) == cudaSuccess ? num_sms(dev) : 148;
+  return s.ctas <= kGemvMinB * sms;
+}
+
+// Tensor maps over the packed tiles for one CTA's box: the codes as a 4-D
+// array [channel block][k tile][chunk][128 rows x 16 bytes] (box: R rows x 4
+// chunks x KR k tiles), the (s_u8, a) pairs as a 3-D array [channel block]
+// [k tile][128 rows x 4 bytes] starting 8192 bytes into each tile.  Boxes
+// past the last k tile are zero-filled; those k tiles are never used.
+bool make_gemv_maps(const uint8_t* tiles, int n_pad, int kt_total, CUtensorMap* codes,
+                    CUtensorMap* prm) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t nblk = (cuuint64_t)(n_pad / kTileN);
+  const cuuint64_t tile = kTileBytes, block = (cuuint64_t)kt_total * kTileBytes;
+  {
+    cuuint64_t dims[4] = {(cuuint64_t)kTileN * 16, 4, (cuuint64_t)kt_total, nblk};
+    cuuint64_t strides[3] = {(cuuint64_t)kTileN * 16, tile, block};
+    cuuint32_t box[4] = {(cuuint32_t)(kGemvR * 16), 4, (cuuint32_t)GemvC::kKR, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (fn(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(tiles), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)kTileN * 4, (cuuint64_t)kt_total, nblk};
+    cuuint64_t strides[2] = {tile, block};
+    cuuint32_t box[3] = {(cuuint32_t)(kGemvR * 4), (cuuint32_t)GemvC::kKR, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(prm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(tiles) + kCodeBytes,
+           dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+// MMA: the warp-MMA kernel (the library's decode form), else the dp4a one
+// (ablation).
+template <bool MMA, bool FUSED>
+cudaError_t launch_gemv(const GemvParams& p, const GemvSchedule& s, const uint8_t* tiles,
+                        int n_pad, cudaStream_t st, bool pdl) {
+  auto k = MMA ? w4a8_gemv_mma_kernel<GemvC::kKR, kGemvMinB, FUSED>
+               : w4a8_gemv_kernel<kGemvR, kGemvP, kGemvMinB, FUSED>;
+  const int smem_max = MMA ? GemvMmaC::smem_bytes(kGemvMaxM) : GemvC::smem_bytes(kGemvMaxM);
+  const int smem = MMA ? GemvMmaC::smem_bytes(p.M) : GemvC::smem_bytes(p.M);
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_relaxed);
+  }
+  CUtensorMap codes, prm;
+  if (!make_gemv_maps(tiles, n_pad, p.kt_total, &codes, &prm)) return cudaErrorInvalidValue;
+  return launch_k(k, dim3(s.ctas), dim3(kGemvThreads), smem, st, pdl, s.splits, codes, prm, p);
+}
+
+// The decode form of a dense call (X fp32 when fused, else Xq / s_x); mma
+// picks the warp-MMA kernel, else the dp4a one.
+int gemm_gemv(const int8_t* Xq, const float* X, const float* s_x, const void* packed, int M,
+              int N, int K, uint16_t* Y, int32_t* acc, bool pdl, void* stream, bool mma = true) {
+  GemvSchedule s;
+  const bool fused = X != nullptr;
+  if (!gemv_schedule(M, N, K, fused, &s)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  const int n_pad = round_up(N, kTileN);
+  GemvParams p;
+  p.Xq = Xq;
+  p.X = X;
+  p.s_x = s_x;
+  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
+  p.hdr = reinterpret_cast<const PackedHeader*>(base);
+  p.Y = Y;
+  p.acc = Y ? nullptr : acc;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.kt_total = K / kTileK;
+  p.splits = s.splits;
+  p.kt_per = s.kt_per;
+  p.wait_limit_ns = wait_budget();
+  const uint8_t* tiles = base + tiles_offset_bytes(n_pad);
+  cudaStream_t st = as_stream(stream);
+  const cudaError_t e =
+      mma ? (fused ? launch_gemv<true, true>(p, s, tiles, n_pad, st, pdl)
+                   : launch_gemv<true, false>(p, s, tiles, n_pad, st, pdl))
+          : (fused ? launch_gemv<false, true>(p, s, tiles, n_pad, st, pdl)
+                   : launch_gemv<false, false>(p, s, tiles, n_pad, st, pdl));
+  return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
 // Grouped (mixture-of-experts) form of a call; groups == 0 for a dense GEMM.
 struct Groups {
   int groups = 0;
@@ -421,12 +577,22 @@ struct Groups {
 
 // W4A8 GEMM, dense (M rows) or grouped (g.m_total rows in g.groups groups of
 // at most M rows each).
+// Kernel paths of a dense call: the library's choice, or one forced (the
+// tensor-core kernel, or the CUDA-core decode form).
+enum class Path { kAuto, kTensor, kWarpMma, kDp4a };
+
 int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
                 int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream,
-                const Groups& g = Groups()) {
+                const Groups& g = Groups(), Path path = Path::kAuto) {
   const int rc = check_common(Xq, s_x, packed, M, N, K, Y, acc, flags);
   if (rc != W4A8_OK || M == 0) return rc;
   const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
+  if (flags & W4A8_FLAG_TENSOR_CORE) path = Path::kTensor;
+  if (g.groups == 0 && path == Path::kDp4a)
+    return gemm_gemv(Xq, nullptr, s_x, packed, M, N, K, Y, acc, pdl, stream, false);
+  if (g.groups == 0 &&
+      (path == Path::kWarpMma || (path == Path::kAuto && prefer_gemv(M, N, K))))
+    return gemm_gemv(Xq, nullptr, s_x, packed, M, N, K, Y, acc, pdl, stream, true);
   const int dev = current_device();
   if (dev < 0) return W4A8_ERR_CUDA;
   const Schedule s = g.groups > 0 ? choose_grouped_schedule(g.groups, g.m_total, M, N, K,
@@ -507,6 +673,7 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
 int gemm_w8_common(const int8_t* Xq, const float* s_x, const int8_t* Wq, const float* s_w,
                    int M, int N, int K, uint16_t* Y, int32_t* acc, unsigned flags,
                    void* stream) {
+  if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;  // (one kernel only)
   const int rc = check_common(Xq, s_x, Wq, M, N, K, Y, acc, flags);
   if (rc != W4A8_OK || M == 0) return rc;
   if (Y && !s_w) return W4A8_ERR_INVALID_ARG;
@@ -546,10 +713,19 @@ int gemm_w8_common(const int8_t* Xq, const float* s_x, const int8_t* Wq, const f
 // reduction; the library's schedule).
 int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* packed, int M,
                  int N, int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
-  if (variant < W4A8_VARIANT_DEFAULT || variant > W4A8_VARIANT_CTA_PAIR)
+  if (variant < W4A8_VARIANT_DEFAULT || variant > W4A8_VARIANT_WARP_MMA)
     return W4A8_ERR_INVALID_ARG;
   if (variant == W4A8_VARIANT_DEFAULT)
     return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream);
+  if (variant == W4A8_VARIANT_TENSOR_CORE)
+    return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream, Groups(), Path::kTensor);
+  if (variant == W4A8_VARIANT_DP4A || variant == W4A8_VARIANT_WARP_MMA) {
+    const int rc0 = check_common(Xq, s_x, packed, M, N, K, Y, acc, flags);
+    if (rc0 != W4A8_OK || M == 0) return rc0;
+    if (!gemv_schedule(M, N, K, false, nullptr)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream, Groups(),
+                       variant == W4A8_VARIANT_DP4A ? Path::kDp4a : Path::kWarpMma);
+  }
   const int rc = check_common(Xq, s_x, packed, M, N, K, Y, acc, flags);
   if (rc != W4A8_OK || M == 0) return rc;
   const bool pdl = (flags & W4A8_FLAG_PDL) != 0;
@@ -622,7 +798,7 @@ bool fused_schedule(int M, int N, int K, int sms, Schedule* out) {
 
 int gemm_fused(const float* X, const void* packed, int M, int N, int K, uint16_t* Y,
                unsigned flags, void* stream) {
-  if (flags & ~(unsigned)W4A8_FLAG_PDL) return W4A8_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)(W4A8_FLAG_PDL | W4A8_FLAG_TENSOR_CORE)) return W4A8_ERR_INVALID_ARG;
   if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
   if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return W4A8_OK;
@@ -630,6 +806,12 @@ int gemm_fused(const float* X, const void* packed, int M, int N, int K, uint16_t
   if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 2)) return W4A8_ERR_MISALIGNED;
   const int dev = current_device();
   if (dev < 0) return W4A8_ERR_CUDA;
+  // a few tokens with whole rows per CTA: the CUDA-core form quantizes in
+  // each CTA; otherwise the tensor-core form with its quantizing warps
+  if (!(flags & W4A8_FLAG_TENSOR_CORE) && gemv_schedule(M, N, K, true, nullptr) &&
+      gemv_env() != 0)
+    return gemm_gemv(nullptr, X, nullptr, packed, M, N, K, Y, nullptr,
+                     (flags & W4A8_FLAG_PDL) != 0, stream);
   Schedule s;
   if (!fused_schedule(M, N, K, num_sms(dev), &s)) return W4A8_ERR_UNSUPPORTED_SHAPE;
   GemmParams p = make_params(s, reinterpret_cast<const float*>(X), M, N, K, Y, nullptr);
@@ -762,6 +944,13 @@ int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K, int
 int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits, int* ctas) {
   if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
   if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  GemvSchedule gs;
+  if (M > 0 && prefer_gemv(M, N, K) && gemv_schedule(M, N, K, false, &gs)) {
+    if (tile_tokens) *tile_tokens = M;
+    if (splits) *splits = gs.splits;
+    if (ctas) *ctas = gs.ctas;
+    return W4A8_OK;
+  }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
   const Schedule s = choose_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev), false);
@@ -769,6 +958,12 @@ int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits, int* 
   if (splits) *splits = s.splits;
   if (ctas) *ctas = s.ctas;
   return W4A8_OK;
+}
+
+int w4a8_gemm_kernel_kind(int M, int N, int K) {
+  if (M < 0 || N < 1 || K < 1) return W4A8_ERR_INVALID_ARG;
+  if (K % kTileK != 0 || K > 65536) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  return M > 0 && prefer_gemv(M, N, K) ? W4A8_KERNEL_WARP_MMA : W4A8_KERNEL_TENSOR_CORE;
 }
 
 int w4a8_grouped_gemm(const int8_t* Xq, const float* s_x, const void* packed, int groups,
@@ -827,7 +1022,10 @@ int w4a8_gemm_fused(const float* X, const void* packed, int M, int N, int K, uin
 int w4a8_gemm_fused_supported(int M, int N, int K) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
-  return fused_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev), nullptr) ? 1 : 0;
+  return (gemv_schedule(M, N, K, true, nullptr) && gemv_env() != 0) ||
+                 fused_schedule(M, N, K, dev < 0 ? 148 : num_sms(dev), nullptr)
+             ? 1
+             : 0;
 }
 
 int w8a8_quantize_weights(const float* W, int N, int K, int8_t* Wq, float* s_w, void* stream) {
@@ -865,6 +1063,12 @@ int w4a8_get_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return W4A8_ERR_CUDA;
   if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return W4A8_ERR_CUDA;
   return v;
+}
+
+int w4a8_debug_set_wait_budget(long long ns) {
+  if (ns < -1 || ns > 10000000000ll) return W4A8_ERR_INVALID_ARG;
+  g_wait_budget.store(ns, std::memory_order_relaxed);
+  return W4A8_OK;
 }
 
 int w4a8_debug_timeout_probe(long long limit_ns, void* stream) {

@@ -148,6 +148,14 @@ int w4a8_gemm(const int8_t* Xq, const float* s_x, const void* packed, int M,
  */
 #define W4A8_FLAG_PDL 1u
 
+/*
+ * W4A8_FLAG_TENSOR_CORE (w4a8_gemm_ex, w4a8_gemm_fused): run the
+ *   tcgen05 kernel even where the library would take the decode form for a
+ *   few tokens (w4a8_gemm_kernel_kind).  The result is
+ *   bit-identical either way; the flag exists to compare and test the two.
+ */
+#define W4A8_FLAG_TENSOR_CORE 2u
+
 /* w4a8_gemm with launch options (flags as above; 0 = w4a8_gemm). */
 int w4a8_gemm_ex(const int8_t* Xq, const float* s_x, const void* packed, int M,
                  int N, int K, uint16_t* Y, unsigned flags, void* stream);
@@ -170,6 +178,22 @@ int w4a8_gemm_i32(const int8_t* Xq, const void* packed, int M, int N, int K,
  */
 int w4a8_gemm_schedule(int M, int N, int K, int* tile_tokens, int* splits,
                        int* ctas);
+
+/*
+ * Which kernel w4a8_gemm / w4a8_gemm_i32 run for a shape (host-only):
+ *   W4A8_KERNEL_TENSOR_CORE  tcgen05 INT8 MMAs, weights dequantized into
+ *                            tensor memory (lead; key_machinery)
+ *   W4A8_KERNEL_WARP_MMA     the decode form for a few tokens: the same
+ *                            IMAD + XOR dequantization (key_machinery) into
+ *                            registers and warp-level INT8 tensor-core MMAs
+ *                            (mma.sync) with INT32 accumulators, 16 output
+ *                            channels per CTA; w4a8_gemm_schedule then
+ *                            reports tile_tokens = M
+ * Both give bit-identical results.  Negative status for a bad shape.
+ */
+#define W4A8_KERNEL_TENSOR_CORE 0
+#define W4A8_KERNEL_WARP_MMA 1
+int w4a8_gemm_kernel_kind(int M, int N, int K);
 
 /*
  * ---- Activation quantization fused into the GEMM (decode) ----
@@ -226,6 +250,15 @@ int w4a8_gemm_fused_supported(int M, int N, int K);
  *                     number of 128-channel blocks (else
  *                     W4A8_ERR_UNSUPPORTED_SHAPE).  The default uses this
  *                     form wherever it applies.
+ *   TENSOR_CORE       the tcgen05 kernel in the library's schedule for
+ *                     every M (the default takes the decode form below for
+ *                     a few tokens)
+ *   WARP_MMA          the decode form (w4a8_gemm_kernel_kind): 16 output
+ *                     channels per CTA, weights dequantized into registers,
+ *                     warp-level INT8 MMAs (mma.sync m16n8k32); 1 <= M <= 8,
+ *                     K <= 32768 (else W4A8_ERR_UNSUPPORTED_SHAPE)
+ *   DP4A              the decode form with CUDA-core 4-way dot products
+ *                     (dp4a) instead of warp MMAs; same limits
  * DEFAULT is the library's own choice (w4a8_gemm_ex / w4a8_gemm_i32).
  * Exactly one of Y (bf16, with s_x) or acc (INT32) is non-NULL.  Other
  * arguments as for w4a8_gemm_ex.
@@ -237,6 +270,9 @@ int w4a8_gemm_fused_supported(int M, int N, int K);
 #define W4A8_VARIANT_ONE_GROUP 4
 #define W4A8_VARIANT_GROUP_ISSUES_MMA 5
 #define W4A8_VARIANT_CTA_PAIR 6
+#define W4A8_VARIANT_TENSOR_CORE 7
+#define W4A8_VARIANT_DP4A 8
+#define W4A8_VARIANT_WARP_MMA 9
 
 int w4a8_gemm_variant(int variant, const int8_t* Xq, const float* s_x,
                       const void* packed, int M, int N, int K, uint16_t* Y,
@@ -331,6 +367,19 @@ int w4a8_get_status(void* stream);
  * status word and returns; nothing faults or hangs.
  */
 int w4a8_debug_timeout_probe(long long limit_ns, void* stream);
+
+/*
+ * Test aid for the GEMM's own failure path: the budget, in nanoseconds, of
+ * the main-loop waits of every kernel launched afterwards by this process
+ * (all entry points, all devices).  -1 restores the default of 2 s; 0 makes
+ * every such wait expire at once, so each launch runs its abort path: the
+ * status word records W4A8_ERR_TIMEOUT, nothing is stored, and the kernel
+ * first waits (always with the full 2 s budget) for the copies, MMAs and
+ * remote adds it already started, then frees its tensor memory and returns.
+ * Valid range -1 .. 1e10; otherwise W4A8_ERR_INVALID_ARG.  Host-only; the
+ * setting is read when a call launches its kernel.
+ */
+int w4a8_debug_set_wait_budget(long long ns);
 
 #ifdef __cplusplus
 }

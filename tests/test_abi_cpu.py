@@ -74,7 +74,8 @@ def test_argument_checks_before_any_launch(L):
     assert L.w4a8_gemm(None, None, None, -1, 128, 256, None, st) == w4.ERR_INVALID_ARG
     assert L.w4a8_gemm(None, None, None, 0, 128, 256, None, st) == w4.OK
     assert L.w4a8_gemm_i32(None, None, 0, 128, 256, None, st) == w4.OK
-    assert L.w4a8_gemm_ex(None, None, None, 0, 128, 256, None, 2, st) == w4.ERR_INVALID_ARG
+    assert L.w4a8_gemm_ex(None, None, None, 0, 128, 256, None, 4, st) == w4.ERR_INVALID_ARG
+    assert L.w4a8_gemm_ex(None, None, None, 0, 128, 256, None, 3, st) == w4.OK  # PDL | TENSOR_CORE
     assert L.w4a8_gemm(None, None, None, 4, 128, 65536 + 128, None, st) == w4.ERR_UNSUPPORTED_SHAPE
     assert L.w4a8_quantize_act(None, 3, 100, None, None, st) == w4.ERR_UNSUPPORTED_SHAPE
     assert L.w4a8_quantize_act(None, 0, 128, None, None, st) == w4.OK
@@ -85,6 +86,7 @@ def test_argument_checks_before_any_launch(L):
     assert L.w8a8_gemm(None, None, None, None, 4, 128, 200, None, 0, st) == w4.ERR_UNSUPPORTED_SHAPE
     assert L.w8a8_gemm(None, None, None, None, 0, 128, 256, None, 0, st) == w4.OK
     assert L.w8a8_gemm(None, None, None, None, 0, 128, 256, None, 4, st) == w4.ERR_INVALID_ARG
+    assert L.w8a8_gemm(None, None, None, None, 0, 128, 256, None, 2, st) == w4.ERR_INVALID_ARG
     assert L.w8a8_gemm(None, None, None, None, 4, 128, 256, None, 0, st) == w4.ERR_INVALID_ARG
     assert L.w8a8_gemm_i32(None, None, 0, 128, 256, None, st) == w4.OK
     assert L.w8a8_quantize_weights(None, 128, 200, None, None, st) == w4.ERR_UNSUPPORTED_SHAPE
@@ -92,13 +94,16 @@ def test_argument_checks_before_any_launch(L):
 
 
 def test_schedule_covers_the_machine(L):
-    # without a device the library assumes 148 SMs
-    T, splits, ctas = w4.w4a8_gemm_schedule(1, 4096, 4096)
-    assert T == 16 and splits > 1 and ctas >= 148
+    # without a device the library assumes 148 SMs; (the tensor-core
+    # kernel's schedule: the dp4a form takes M <= 4, checked below)
+    T, splits, ctas = w4.w4a8_gemm_schedule(16, 4096, 4096)
+    assert T == 16 and splits > 1 and ctas >= 128
     T, splits, ctas = w4.w4a8_gemm_schedule(8192, 8192, 8192)
     assert T == 256 and splits == 1 and ctas == 64 * 32
     for M in (1, 2, 16, 17, 32, 33, 64, 65, 128, 129, 256, 257, 4096):
         for N, K in ((4096, 4096), (28672, 8192), (8192, 28672), (128, 65536)):
+            if w4.w4a8_gemm_kernel_kind(M, N, K) != w4.KERNEL_TENSOR_CORE:
+                continue
             T, splits, ctas = w4.w4a8_gemm_schedule(M, N, K)
             assert T >= min(M, 16) and T in (16, 32, 64, 128, 256)
             assert 1 <= splits <= 8                    # one portable cluster
@@ -137,10 +142,44 @@ def test_fused_call_shape_rules(L):
     # (up to 16 tokens, a k range per CTA that stays resident, and the CTA's
     # slice of X within the quantizing warps' registers); everything else is
     # refused before any launch
-    ok = [(1, 4096, 4096), (4, 4096, 4096), (4, 28672, 512), (16, 28672, 128)]
-    refused = [(0, 4096, 4096), (8, 4096, 4096), (16, 4096, 4096), (17, 256, 4096),
-               (16, 28672, 768), (1, 4096, 4000)]
+    ok = [(1, 4096, 4096), (4, 4096, 4096), (4, 28672, 512), (16, 28672, 128),
+          (8, 4096, 4096)]  # (the last: the CUDA-core form, whole rows per CTA)
+    refused = [(0, 4096, 4096), (16, 4096, 4096), (17, 256, 4096),
+               (16, 28672, 768), (1, 4096, 4000), (8, 4096, 8192)]
     for sh in ok:
         assert w4.w4a8_gemm_fused_supported(*sh), sh
     for sh in refused:
         assert not w4.w4a8_gemm_fused_supported(*sh), sh
+
+
+def test_kernel_kind_and_decode_schedule(L):
+    """Host-only: a few tokens take the decode (warp-MMA) form with 16 output
+    channels per CTA and split-K clusters of at most 8 for rows longer than
+    4096; everything else the tensor-core kernel."""
+    # (without a device the library assumes 148 SMs: the decode form when its
+    # CTAs fit two per SM)
+    assert w4.w4a8_gemm_kernel_kind(1, 4096, 4096) == w4.KERNEL_WARP_MMA      # 256 CTAs
+    assert w4.w4a8_gemm_kernel_kind(8, 4096, 4096) == w4.KERNEL_WARP_MMA
+    assert w4.w4a8_gemm_kernel_kind(9, 4096, 4096) == w4.KERNEL_TENSOR_CORE
+    assert w4.w4a8_gemm_kernel_kind(1, 12288, 4096) == w4.KERNEL_TENSOR_CORE  # 768 CTAs
+    assert w4.w4a8_gemm_kernel_kind(4, 2048, 8192) == w4.KERNEL_WARP_MMA      # 2 splits
+    assert w4.w4a8_gemm_kernel_kind(64, 4096, 4096) == w4.KERNEL_TENSOR_CORE
+    assert w4.w4a8_gemm_kernel_kind(1, 128, 65536) == w4.KERNEL_TENSOR_CORE  # 16 splits
+    assert w4.w4a8_gemm_kernel_kind(0, 4096, 4096) == w4.KERNEL_TENSOR_CORE
+    assert L.w4a8_gemm_kernel_kind(1, 4096, 200) == w4.ERR_UNSUPPORTED_SHAPE
+    assert L.w4a8_gemm_kernel_kind(-1, 4096, 256) == w4.ERR_INVALID_ARG
+    # schedule of the decode form: tile = all M tokens, splits, CTAs
+    assert w4.w4a8_gemm_schedule(1, 4096, 4096) == (1, 1, 256)
+    assert w4.w4a8_gemm_schedule(2, 1024, 11008) == (2, 3, 192)
+    assert w4.w4a8_gemm_schedule(3, 200, 384) == (3, 1, 16)  # N padded to 256
+    assert w4.VARIANTS["tensor_core"] == 7 and w4.VARIANTS["dp4a"] == 8
+    assert w4.VARIANTS["warp_mma"] == 9
+
+
+def test_debug_wait_budget_range(L):
+    """Host-only: the test wait budget accepts -1 (default), 0 .. 1e10 ns."""
+    assert L.w4a8_debug_set_wait_budget(-2) == w4.ERR_INVALID_ARG
+    assert L.w4a8_debug_set_wait_budget(10000000001) == w4.ERR_INVALID_ARG
+    assert L.w4a8_debug_set_wait_budget(0) == w4.OK
+    assert L.w4a8_debug_set_wait_budget(5000) == w4.OK
+    assert L.w4a8_debug_set_wait_budget(-1) == w4.OK

@@ -40,14 +40,18 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("core", ["library", "tensor_core"])
 @pytest.mark.parametrize("M,N,K,kind", CASES)
-def test_fused_matches_two_calls_and_oracle(M, N, K, kind):
+def test_fused_matches_two_calls_and_oracle(M, N, K, kind, core):
+    """``library``: the library's choice (the CUDA-core form where it applies);
+    ``tensor_core``: the tensor-core fused kernel forced by its flag."""
     assert w4.w4a8_gemm_fused_supported(M, N, K), (M, N, K, w4.w4a8_gemm_schedule(M, N, K))
     X = wl.random_matrix(M, K, 8000 + M + K, std=1.0, kind=kind)
     W = wl.random_matrix(N, K, 9000 + N + K, std=0.02)
     pk = w4.w4a8_quantize_weights(W.cuda())
     Xd = X.cuda()
-    Y = w4.w4a8_gemm_fused(Xd, pk, flags=w4.W4A8_FLAG_PDL)
+    flags = w4.W4A8_FLAG_PDL | (w4.W4A8_FLAG_TENSOR_CORE if core == "tensor_core" else 0)
+    Y = w4.w4a8_gemm_fused(Xd, pk, flags=flags)
     torch.cuda.synchronize()
     assert w4.w4a8_get_status() == 0
     Xq, sx = w4.w4a8_quantize_act(Xd)
@@ -87,11 +91,19 @@ def test_fused_codes_at_rounding_boundaries(absmax):
 def test_fused_unsupported_shapes_are_rejected_before_launch():
     W = wl.random_matrix(256, 4096, 1, std=0.02).cuda()
     pk = w4.w4a8_quantize_weights(W)
-    # 17 and 64 tokens: past the 16-token tile; 8 and 16 tokens over 4096
-    # k: the CTA's slice of X would not fit the quantizing warps' registers
-    for M in (17, 64, 8, 16):
+    # 17 and 64 tokens: past the 16-token tile; 16 tokens over 4096 k: the
+    # CTA's slice of X would not fit the quantizing warps' registers (and
+    # the CUDA-core form takes at most 8 tokens)
+    for M in (17, 64, 16):
         assert not w4.w4a8_gemm_fused_supported(M, 256, 4096)
         with pytest.raises(w4.W4A8Error) as e:
             w4.w4a8_gemm_fused(torch.zeros(M, 4096, device="cuda"), pk)
         assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
+    # 8 tokens over 4096 k: the CUDA-core form only (the tensor-core fused
+    # kernel refuses it)
+    assert w4.w4a8_gemm_fused_supported(8, 256, 4096)
+    with pytest.raises(w4.W4A8Error) as e:
+        w4.w4a8_gemm_fused(torch.zeros(8, 4096, device="cuda"), pk,
+                           flags=w4.W4A8_FLAG_TENSOR_CORE)
+    assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
     assert w4.w4a8_get_status() == 0

@@ -59,7 +59,7 @@ def test_variant_parity(variant, M, N, K, kind):
 def test_variant_rejections():
     L = w4.lib()
     st = torch.cuda.current_stream().cuda_stream
-    assert L.w4a8_gemm_variant(9, None, None, None, 0, 128, 256, None, None, 0, st) == w4.ERR_INVALID_ARG
+    assert L.w4a8_gemm_variant(10, None, None, None, 0, 128, 256, None, None, 0, st) == w4.ERR_INVALID_ARG
     x = torch.zeros(4, dtype=torch.int32, device="cuda")
     assert L.w4a8_gemm_variant(1, None, None, None, 1, 128, 256, x.data_ptr(), x.data_ptr(), 0, st) == w4.ERR_INVALID_ARG
 
