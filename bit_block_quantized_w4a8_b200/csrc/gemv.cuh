@@ -331,9 +331,12 @@ __global__ void __launch_bounds__(kGemvThreads, MINB)
 // Warp w takes the chunks q = w + 8 i of the CTA's 4 KR chunks (k tile
 // q / 4, chunk q % 4); the eight warps' 16 x 8 partial tiles are added
 // through shared memory.  Tokens past M read zeros.
+constexpr int kGemvMmaMaxM = 16;  // two groups of 8 tokens (the MMA's N)
+
 template <int KR>
 struct GemvMmaCfg {
   static constexpr int kR = 16;
+  static constexpr int kMaxM = kGemvMmaMaxM;
   static constexpr int kWarps = kGemvThreads / 32;
   static constexpr int kChunks = 4 * KR;
   static constexpr int kCpw = kChunks / kWarps;  // chunks per warp
@@ -341,13 +344,16 @@ struct GemvMmaCfg {
   static constexpr int kCodeBytes = KR * 4 * kR * 16;
   static constexpr int kPrmBytes = KR * kR * 4;
   static constexpr int kOffPrm = kCodeBytes;
-  static constexpr int kOffRed = (kOffPrm + kPrmBytes + 127) & ~127;  // [warp][row][8] int32
-  static constexpr int kRedBytes = kWarps * kR * 8 * 4;
+  // [warp][m][row] int32, rows padded to 17 (fragment stores and the
+  // owners' reads both spread over the banks)
+  static constexpr int kRedStride = kR + 1;
+  static constexpr int kOffRed = (kOffPrm + kPrmBytes + 127) & ~127;
+  static constexpr int kRedBytes = kWarps * kMaxM * kRedStride * 4;
   static constexpr int kOffRecv = kOffRed + kRedBytes;  // split-K: [m][row] int32
-  static constexpr int kOffSx = kOffRecv + kGemvMaxM * kR * 4;  // [m] fp32
-  static constexpr int kOffSw = kOffSx + 4 * kGemvMaxM;           // [row] fp32
-  static constexpr int kOffAmax = kOffSw + 4 * kR;                // FUSED: [warp][m] fp32
-  static constexpr int kOffBar = (kOffAmax + 4 * kWarps * kGemvMaxM + 7) & ~7;
+  static constexpr int kOffSx = kOffRecv + kMaxM * kR * 4;  // [m] fp32
+  static constexpr int kOffSw = kOffSx + 4 * kMaxM;           // [row] fp32
+  static constexpr int kOffAmax = kOffSw + 4 * kR;            // FUSED: [warp][m] fp32
+  static constexpr int kOffBar = (kOffAmax + 4 * kWarps * kMaxM + 7) & ~7;
   static constexpr int kOffMisc = kOffBar + 3 * 8;
   static constexpr int kOffX = (kOffMisc + 16 + 127) & ~127;
   // activation rows padded by 16 bytes: the 8 tokens of a B fragment load
@@ -372,7 +378,9 @@ __device__ __forceinline__ uint32_t dequant_word(uint32_t w, uint32_t sh, uint32
   return (((w >> sh) & 0x0F0F0F0Fu) * s + a4) ^ 0x80808080u;
 }
 
-template <int KR, int MINB, bool FUSED>
+// NG: token groups of 8 (1 for M <= 8, 2 for M <= 16); a group's MMAs run
+// whatever M is (tokens past M have zero B fragments).
+template <int KR, int NG, int MINB, bool FUSED>
 __global__ void __launch_bounds__(kGemvThreads, MINB)
     w4a8_gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes,
                          const __grid_constant__ CUtensorMap tm_prm, const GemvParams p) {
@@ -474,38 +482,62 @@ __global__ void __launch_bounds__(kGemvThreads, MINB)
     if (tid == 32) hdr_ok = p.hdr->magic == kMagic && p.hdr->N == p.N && p.hdr->K == p.K;
     float* amax_s = reinterpret_cast<float*>(smem + C::kOffAmax);  // [warp][m]
     const int n4 = nk * (kTileK / 4);
+    // float4 f = tid + 256 j of a token row (at most kF4 per thread): every
+    // load of a token is issued before any is used (one L2 round trip, not
+    // one per float4)
+    constexpr int kF4 = KR * (kTileK / 4) / kGemvThreads;
 #pragma unroll
-    for (int m = 0; m < kGemvMaxM; ++m) {
+    for (int m = 0; m < 8 * NG; ++m) {
       if (m < M) {
         const float4* xr = reinterpret_cast<const float4*>(p.X + (size_t)m * p.K + k_lo);
+        float4 v[kF4];
+#pragma unroll
+        for (int j = 0; j < kF4; ++j) {
+          const int f = tid + kGemvThreads * j;
+          v[j] = f < n4 ? __ldg(xr + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         float am = 0.0f;
-        for (int f = tid; f < n4; f += kGemvThreads) am = fmaxf(am, absmax4(__ldg(xr + f)));
+#pragma unroll
+        for (int j = 0; j < kF4; ++j) am = fmaxf(am, absmax4(v[j]));
         am = warp_max(am);
-        if (lane == 0) amax_s[warp * kGemvMaxM + m] = am;
+        if (lane == 0) amax_s[warp * C::kMaxM + m] = am;
       }
     }
     __syncthreads();
     if (tid < M) {
       float am = 0.0f;
 #pragma unroll
-      for (int w = 0; w < C::kWarps; ++w) am = fmaxf(am, amax_s[w * kGemvMaxM + tid]);
+      for (int w = 0; w < C::kWarps; ++w) am = fmaxf(am, amax_s[w * C::kMaxM + tid]);
       sx_s[tid] = __fdiv_rn(am, 127.0f);
     }
     __syncthreads();
     uint8_t* xw = smem + C::kOffX;
 #pragma unroll
-    for (int m = 0; m < kGemvMaxM; ++m) {
+    for (int m = 0; m < 8 * NG; ++m) {
       if (m < M) {
         const float4* xr = reinterpret_cast<const float4*>(p.X + (size_t)m * p.K + k_lo);
         const float s = sx_s[m];
         uint8_t* xm = xw + m * C::kXStride;
+        // (the row is read again: an L1 hit)
+        float4 v[kF4];
+#pragma unroll
+        for (int j = 0; j < kF4; ++j) {
+          const int f = tid + kGemvThreads * j;
+          v[j] = f < n4 ? __ldg(xr + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         if (rcp_quant_ok(s)) {  // (uniform: one scale per token)
           const float y = __fdiv_rn(1.0f, s);
-          for (int f = tid; f < n4; f += kGemvThreads)
-            *reinterpret_cast<uint32_t*>(xm + 4 * f) = quant4_rcp(__ldg(xr + f), s, y);
+#pragma unroll
+          for (int j = 0; j < kF4; ++j) {
+            const int f = tid + kGemvThreads * j;
+            if (f < n4) *reinterpret_cast<uint32_t*>(xm + 4 * f) = quant4_rcp(v[j], s, y);
+          }
         } else {
-          for (int f = tid; f < n4; f += kGemvThreads)
-            *reinterpret_cast<uint32_t*>(xm + 4 * f) = quant4(__ldg(xr + f), s);
+#pragma unroll
+          for (int j = 0; j < kF4; ++j) {
+            const int f = tid + kGemvThreads * j;
+            if (f < n4) *reinterpret_cast<uint32_t*>(xm + 4 * f) = quant4(v[j], s);
+          }
         }
       }
     }
@@ -522,35 +554,47 @@ __global__ void __launch_bounds__(kGemvThreads, MINB)
   // of those chunks are zero too).  A runtime branch around the
   // warp-collective mma.sync, uniform or not, measured about 140 cycles per
   // chunk on this GPU (the loop took 2900 cycles instead of 670).  All B
-  // fragments are read first; two accumulator sets halve the MMA chain.
-  int32_t d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+  // fragments are read with select, not under a branch; two accumulator
+  // sets halve the MMA chain.
+  // accumulator chains: two per group of one (independent chains halve the
+  // MMA latency chain), one per group of two (the groups interleave)
+  constexpr int ND = NG == 1 ? 2 : NG;
+  int32_t d[ND][4];
+#pragma unroll
+  for (int j = 0; j < ND; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0;
   if (live) {
-    const bool tok = g < M;
-    const uint8_t* xg = smem + C::kOffX + (tok ? g : 0) * C::kXStride + 4 * t;
-    uint32_t b[C::kCpw][2];
+    const uint8_t* xg[NG];
+    bool tok[NG];
+#pragma unroll
+    for (int gr = 0; gr < NG; ++gr) {
+      const int tk = 8 * gr + g;  // this lane's token in group gr
+      tok[gr] = tk < M;
+      xg[gr] = smem + C::kOffX + (tok[gr] ? tk : 0) * C::kXStride + 4 * t;
+    }
 #pragma unroll
     for (int i = 0; i < C::kCpw; ++i) {
       const int q = warp + C::kWarps * i, kt = q >> 2, c = q & 3;
-      const bool use = tok && kt < nk;
-      const uint8_t* xp = xg + kt * kTileK + c * 32;  // inside the buffer for kt < KR
-      b[i][0] = use ? *reinterpret_cast<const uint32_t*>(xp) : 0u;
-      b[i][1] = use ? *reinterpret_cast<const uint32_t*>(xp + 16) : 0u;
-    }
 #pragma unroll
-    for (int i = 0; i < C::kCpw; ++i) {
-      if (i & 1)
-        mma_s8_16x8x32(d1, a[i], b[i][0], b[i][1]);
-      else
-        mma_s8_16x8x32(d0, a[i], b[i][0], b[i][1]);
+      for (int gr = 0; gr < NG; ++gr) {
+        const bool use = tok[gr] && kt < nk;
+        const uint8_t* xp = xg[gr] + kt * kTileK + c * 32;  // inside the buffer for kt < KR
+        const uint32_t b0 = use ? *reinterpret_cast<const uint32_t*>(xp) : 0u;
+        const uint32_t b1 = use ? *reinterpret_cast<const uint32_t*>(xp + 16) : 0u;
+        mma_s8_16x8x32(d[NG == 1 ? (i & 1) : gr], a[i], b0, b1);
+      }
     }
   }
-  // the warps' 16 x 8 partial tiles: red[warp][row][token]
-  {
-    int32_t* rw = red + warp * R * 8;
-    rw[g * 8 + 2 * t] = d0[0] + d1[0];
-    rw[g * 8 + 2 * t + 1] = d0[1] + d1[1];
-    rw[(g + 8) * 8 + 2 * t] = d0[2] + d1[2];
-    rw[(g + 8) * 8 + 2 * t + 1] = d0[3] + d1[3];
+  // the warps' partial tiles: red[warp][token][row]
+  constexpr int RS = C::kRedStride;
+#pragma unroll
+  for (int gr = 0; gr < NG; ++gr) {
+    const int32_t* dd = d[NG == 1 ? 0 : gr];
+    const int32_t* de = NG == 1 ? d[1] : nullptr;
+    int32_t* rw = red + (warp * C::kMaxM + 8 * gr) * RS;
+    rw[(2 * t) * RS + g] = dd[0] + (de ? de[0] : 0);
+    rw[(2 * t + 1) * RS + g] = dd[1] + (de ? de[1] : 0);
+    rw[(2 * t) * RS + g + 8] = dd[2] + (de ? de[2] : 0);
+    rw[(2 * t + 1) * RS + g + 8] = dd[3] + (de ? de[3] : 0);
   }
   __syncthreads();
   int total = 0;
@@ -558,7 +602,7 @@ __global__ void __launch_bounds__(kGemvThreads, MINB)
   const bool owner = tid < M * R;
   if (owner) {
 #pragma unroll
-    for (int w = 0; w < C::kWarps; ++w) total += red[(w * R + orow) * 8 + om];
+    for (int w = 0; w < C::kWarps; ++w) total += red[(w * C::kMaxM + om) * RS + orow];
   }
 
   // ---- split-K: the other splits add their sums into the leader

@@ -434,10 +434,12 @@ struct GemvSchedule {
   int splits = 1, kt_per = 1, ctas = 0;
 };
 
-// Whether the CUDA-core form applies to a shape (fused: one split only, the
-// CTA then holds whole rows of X for the per-token absmax).
-bool gemv_schedule(int M, int N, int K, bool fused, GemvSchedule* out) {
-  if (M < 1 || M > kGemvMaxM || N < 1 || K < kTileK || K % kTileK != 0 || K > 65536)
+// Whether a decode form applies to a shape: up to 16 tokens for the
+// warp-MMA form, 8 for the dp4a one (fused: one split only, the CTA then
+// holds whole rows of X for the per-token absmax).
+bool gemv_schedule(int M, int N, int K, bool fused, GemvSchedule* out, bool mma = true) {
+  const int max_m = mma ? kGemvMmaMaxM : kGemvMaxM;
+  if (M < 1 || M > max_m || N < 1 || K < kTileK || K % kTileK != 0 || K > 65536)
     return false;
   const int kt = K / kTileK;
   const int splits = (kt + GemvC::kKR - 1) / GemvC::kKR;
@@ -512,14 +514,15 @@ bool make_gemv_maps(const uint8_t* tiles, int n_pad, int kt_total, CUtensorMap* 
   return true;
 }
 
-// MMA: the warp-MMA kernel (the library's decode form), else the dp4a one
-// (ablation).
-template <bool MMA, bool FUSED>
+// MMA: the warp-MMA kernel (the library's decode form; NG groups of 8
+// tokens), else the dp4a one (ablation).
+template <bool MMA, int NG, bool FUSED>
 cudaError_t launch_gemv(const GemvParams& p, const GemvSchedule& s, const uint8_t* tiles,
                         int n_pad, cudaStream_t st, bool pdl) {
-  auto k = MMA ? w4a8_gemv_mma_kernel<GemvC::kKR, kGemvMinB, FUSED>
+  auto k = MMA ? w4a8_gemv_mma_kernel<GemvC::kKR, NG, kGemvMinB, FUSED>
                : w4a8_gemv_kernel<kGemvR, kGemvP, kGemvMinB, FUSED>;
-  const int smem_max = MMA ? GemvMmaC::smem_bytes(kGemvMaxM) : GemvC::smem_bytes(kGemvMaxM);
+  const int smem_max =
+      MMA ? GemvMmaC::smem_bytes(8 * NG) : GemvC::smem_bytes(kGemvMaxM);
   const int smem = MMA ? GemvMmaC::smem_bytes(p.M) : GemvC::smem_bytes(p.M);
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
@@ -540,7 +543,7 @@ int gemm_gemv(const int8_t* Xq, const float* X, const float* s_x, const void* pa
               int N, int K, uint16_t* Y, int32_t* acc, bool pdl, void* stream, bool mma = true) {
   GemvSchedule s;
   const bool fused = X != nullptr;
-  if (!gemv_schedule(M, N, K, fused, &s)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (!gemv_schedule(M, N, K, fused, &s, mma)) return W4A8_ERR_UNSUPPORTED_SHAPE;
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   const int n_pad = round_up(N, kTileN);
   GemvParams p;
@@ -560,11 +563,16 @@ int gemm_gemv(const int8_t* Xq, const float* X, const float* s_x, const void* pa
   p.wait_limit_ns = wait_budget();
   const uint8_t* tiles = base + tiles_offset_bytes(n_pad);
   cudaStream_t st = as_stream(stream);
-  const cudaError_t e =
-      mma ? (fused ? launch_gemv<true, true>(p, s, tiles, n_pad, st, pdl)
-                   : launch_gemv<true, false>(p, s, tiles, n_pad, st, pdl))
-          : (fused ? launch_gemv<false, true>(p, s, tiles, n_pad, st, pdl)
-                   : launch_gemv<false, false>(p, s, tiles, n_pad, st, pdl));
+  cudaError_t e;
+  if (!mma)
+    e = fused ? launch_gemv<false, 1, true>(p, s, tiles, n_pad, st, pdl)
+              : launch_gemv<false, 1, false>(p, s, tiles, n_pad, st, pdl);
+  else if (M <= 8)
+    e = fused ? launch_gemv<true, 1, true>(p, s, tiles, n_pad, st, pdl)
+              : launch_gemv<true, 1, false>(p, s, tiles, n_pad, st, pdl);
+  else
+    e = fused ? launch_gemv<true, 2, true>(p, s, tiles, n_pad, st, pdl)
+              : launch_gemv<true, 2, false>(p, s, tiles, n_pad, st, pdl);
   return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
@@ -722,7 +730,8 @@ int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* pa
   if (variant == W4A8_VARIANT_DP4A || variant == W4A8_VARIANT_WARP_MMA) {
     const int rc0 = check_common(Xq, s_x, packed, M, N, K, Y, acc, flags);
     if (rc0 != W4A8_OK || M == 0) return rc0;
-    if (!gemv_schedule(M, N, K, false, nullptr)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if (!gemv_schedule(M, N, K, false, nullptr, variant == W4A8_VARIANT_WARP_MMA))
+      return W4A8_ERR_UNSUPPORTED_SHAPE;
     return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream, Groups(),
                        variant == W4A8_VARIANT_DP4A ? Path::kDp4a : Path::kWarpMma);
   }

@@ -96,8 +96,9 @@ def test_argument_checks_before_any_launch(L):
 def test_schedule_covers_the_machine(L):
     # without a device the library assumes 148 SMs; (the tensor-core
     # kernel's schedule: the dp4a form takes M <= 4, checked below)
-    T, splits, ctas = w4.w4a8_gemm_schedule(16, 4096, 4096)
-    assert T == 16 and splits > 1 and ctas >= 128
+    T, splits, ctas = w4.w4a8_gemm_schedule(16, 28672, 8192)
+    assert w4.w4a8_gemm_kernel_kind(16, 28672, 8192) == w4.KERNEL_TENSOR_CORE
+    assert T == 16 and ctas >= 148
     T, splits, ctas = w4.w4a8_gemm_schedule(8192, 8192, 8192)
     assert T == 256 and splits == 1 and ctas == 64 * 32
     for M in (1, 2, 16, 17, 32, 33, 64, 65, 128, 129, 256, 257, 4096):
@@ -143,9 +144,9 @@ def test_fused_call_shape_rules(L):
     # slice of X within the quantizing warps' registers); everything else is
     # refused before any launch
     ok = [(1, 4096, 4096), (4, 4096, 4096), (4, 28672, 512), (16, 28672, 128),
-          (8, 4096, 4096)]  # (the last: the CUDA-core form, whole rows per CTA)
-    refused = [(0, 4096, 4096), (16, 4096, 4096), (17, 256, 4096),
-               (16, 28672, 768), (1, 4096, 4000), (8, 4096, 8192)]
+          (8, 4096, 4096), (16, 4096, 4096)]  # (the last two: the decode form)
+    refused = [(0, 4096, 4096), (17, 256, 4096), (1, 4096, 4000), (8, 4096, 8192),
+               (16, 4096, 8192)]
     for sh in ok:
         assert w4.w4a8_gemm_fused_supported(*sh), sh
     for sh in refused:
@@ -159,8 +160,8 @@ def test_kernel_kind_and_decode_schedule(L):
     # (without a device the library assumes 148 SMs: the decode form when its
     # CTAs fit two per SM)
     assert w4.w4a8_gemm_kernel_kind(1, 4096, 4096) == w4.KERNEL_WARP_MMA      # 256 CTAs
-    assert w4.w4a8_gemm_kernel_kind(8, 4096, 4096) == w4.KERNEL_WARP_MMA
-    assert w4.w4a8_gemm_kernel_kind(9, 4096, 4096) == w4.KERNEL_TENSOR_CORE
+    assert w4.w4a8_gemm_kernel_kind(16, 4096, 4096) == w4.KERNEL_WARP_MMA
+    assert w4.w4a8_gemm_kernel_kind(17, 4096, 4096) == w4.KERNEL_TENSOR_CORE
     assert w4.w4a8_gemm_kernel_kind(1, 12288, 4096) == w4.KERNEL_TENSOR_CORE  # 768 CTAs
     assert w4.w4a8_gemm_kernel_kind(4, 2048, 8192) == w4.KERNEL_WARP_MMA      # 2 splits
     assert w4.w4a8_gemm_kernel_kind(64, 4096, 4096) == w4.KERNEL_TENSOR_CORE

@@ -51,16 +51,18 @@ def test_abort_path_reports_timeout_stores_nothing_and_context_survives(M, N, K,
     out = torch.full((M, N), 7, dtype=torch.int32, device="cuda")
     torch.cuda.synchronize()
     assert w4.w4a8_get_status() == 0
+    def run(out=None):
+        return w4.w4a8_gemm_variant(variant, Xq, None, pk, i32=True, out=out)
     w4.w4a8_debug_set_wait_budget(0)
     try:
-        w4.w4a8_gemm_variant(variant, Xq, None, pk, i32=True, out=out)
+        run(out)
         status = w4.w4a8_get_status()
     finally:
         w4.w4a8_debug_set_wait_budget(-1)
     assert status == w4.ERR_TIMEOUT, what
     assert int((out != 7).sum()) == 0, what + ": an aborted launch stored outputs"
     # the context is usable and the same call is exact again
-    acc = w4.w4a8_gemm_variant(variant, Xq, None, pk, i32=True)
+    acc = run()
     torch.cuda.synchronize()
     assert w4.w4a8_get_status() == 0
     Xq_ref, sx_ref = oracle.quantize_act(X.numpy())

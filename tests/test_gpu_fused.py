@@ -91,19 +91,18 @@ def test_fused_codes_at_rounding_boundaries(absmax):
 def test_fused_unsupported_shapes_are_rejected_before_launch():
     W = wl.random_matrix(256, 4096, 1, std=0.02).cuda()
     pk = w4.w4a8_quantize_weights(W)
-    # 17 and 64 tokens: past the 16-token tile; 16 tokens over 4096 k: the
-    # CTA's slice of X would not fit the quantizing warps' registers (and
-    # the CUDA-core form takes at most 8 tokens)
-    for M in (17, 64, 16):
+    # 17 and 64 tokens: past the 16-token tile and the decode form's limit
+    for M in (17, 64):
         assert not w4.w4a8_gemm_fused_supported(M, 256, 4096)
         with pytest.raises(w4.W4A8Error) as e:
             w4.w4a8_gemm_fused(torch.zeros(M, 4096, device="cuda"), pk)
         assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
-    # 8 tokens over 4096 k: the CUDA-core form only (the tensor-core fused
-    # kernel refuses it)
-    assert w4.w4a8_gemm_fused_supported(8, 256, 4096)
-    with pytest.raises(w4.W4A8Error) as e:
-        w4.w4a8_gemm_fused(torch.zeros(8, 4096, device="cuda"), pk,
-                           flags=w4.W4A8_FLAG_TENSOR_CORE)
-    assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
+    # 8 and 16 tokens over 4096 k: the decode form only (the tensor-core
+    # fused kernel cannot hold the CTA's slice of X in its registers)
+    for M in (8, 16):
+        assert w4.w4a8_gemm_fused_supported(M, 256, 4096)
+        with pytest.raises(w4.W4A8Error) as e:
+            w4.w4a8_gemm_fused(torch.zeros(M, 4096, device="cuda"), pk,
+                               flags=w4.W4A8_FLAG_TENSOR_CORE)
+        assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
     assert w4.w4a8_get_status() == 0

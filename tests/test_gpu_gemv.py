@@ -39,8 +39,11 @@ CASES = [
     (5, 384, 8192, 128, "normal"),     # group 128, 2 splits
     (6, 136, 11008, 64, "rowzero"),    # 86 k tiles: 3 splits (29, 29, 28), zero rows
     (7, 512, 28672, 64, "normal"),     # 224 k tiles: 7 splits
-    (8, 640, 2048, 64, "heavy"),       # largest M
+    (8, 640, 2048, 64, "heavy"),       # one group of 8 tokens, full
     (8, 8, 32768, 64, "normal"),       # 8 splits (the cluster limit), N < one slice
+    (9, 4096, 4096, 64, "normal"),     # two token groups (warp-MMA form only)
+    (13, 200, 11008, 64, "rowzero"),   # two groups, 3 splits, ragged N
+    (16, 1024, 4096, 128, "ties"),     # largest M, group 128
 ]
 
 
@@ -56,6 +59,8 @@ FORMS = ["warp_mma", "dp4a"]
 @pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("M,N,K,group,kind", CASES)
 def test_decode_form_matches_oracle_and_tensor_core(M, N, K, group, kind, form):
+    if form == "dp4a" and M > 8:
+        pytest.skip("the dp4a form takes at most 8 tokens")
     X, W = _inputs(M, N, K, group, kind, 700 + M + N + K)
     wq = oracle.quantize_weights(W.numpy(), group=group)
     Xq_ref, sx_ref = oracle.quantize_act(X.numpy())
@@ -85,10 +90,10 @@ def test_default_dispatch_uses_the_decode_form_for_few_tokens():
     assert torch.equal(Y.view(torch.int16), Yt.view(torch.int16))
 
 
-@pytest.mark.parametrize("form", FORMS)
-def test_decode_form_refuses_shapes_outside_its_limits(form):
+@pytest.mark.parametrize("form,M", [("warp_mma", 17), ("dp4a", 9)])
+def test_decode_form_refuses_shapes_outside_its_limits(form, M):
     pk = w4.w4a8_quantize_weights(torch.randn(128, 256, device="cuda") * 0.02)
-    Xq = torch.zeros(9, 256, dtype=torch.int8, device="cuda")
+    Xq = torch.zeros(M, 256, dtype=torch.int8, device="cuda")
     with pytest.raises(w4.W4A8Error) as e:
         w4.w4a8_gemm_variant(form, Xq, None, pk, i32=True)
     assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
@@ -114,7 +119,8 @@ def test_decode_pdl_chain_and_repeated_runs(form):
     for K in (4096, 11008):
         W = wl.random_matrix(384, K, 41 + K, std=0.02).cuda()
         pk = w4.w4a8_quantize_weights(W)
-        Xs = [wl.random_matrix(M, K, 50 + M, std=1.0).cuda() for M in (1, 3, 4, 8)]
+        Ms = (1, 3, 4, 8) + ((12, 16) if form == "warp_mma" else ())
+        Xs = [wl.random_matrix(M, K, 50 + M, std=1.0).cuda() for M in Ms]
         torch.cuda.synchronize()
         ref = []
         for X in Xs:
@@ -139,6 +145,8 @@ FUSED_CASES = [
     (4, 200, 512, "rowzero"),
     (8, 1024, 4096, "ties"),
     (3, 256, 128, "normal"),
+    (16, 4096, 4096, "heavy"),
+    (11, 200, 1024, "rowzero"),
 ]
 
 
@@ -184,7 +192,7 @@ def test_fused_decode_form_codes_at_rounding_boundaries():
                                              ("llama7b_like", "down"),
                                              ("llama70b_like", "down")])
 def test_decode_form_full_size_layers(name, layer_name):
-    """The decode layers at full size for M = 1..8 through the warp-MMA
+    """The decode layers at full size for M = 1..16 through the warp-MMA
     decode form: every output element against the oracle."""
     layer = [L for L in wl.WORKLOADS[name].layers if L.name == layer_name][0]
     N, K = layer.N, layer.K
@@ -192,7 +200,7 @@ def test_decode_form_full_size_layers(name, layer_name):
     wq = oracle.quantize_weights(W.numpy())
     pk = w4.w4a8_quantize_weights(W.cuda())
     del W
-    for M in (1, 2, 4, 8):
+    for M in (1, 2, 4, 8, 16):
         X = wl.make_activations(M, K, 1234 + M, 0.01, 20.0)
         Xq_ref, sx_ref = oracle.quantize_act(X.numpy())
         acc_ref, y_ref = oracle.w4a8_gemm(Xq_ref, sx_ref, wq)
