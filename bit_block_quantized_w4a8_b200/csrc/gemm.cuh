@@ -135,15 +135,13 @@ struct GemmCfg {
   static constexpr int kNumBars = (PAIR ? 2 : 3) * SS + 2 * AS + 3 + (FUSED ? 1 : 0);
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kOffSx = kOffMisc + 16;
-  // the tile's 128 channel scales, staged for the split-K reduction
-  static constexpr int kOffSwS = (kOffSx + 4 * T + 15) & ~15;
   // partial tiles of at most kPushMaxM tokens are pushed (remote atomic
   // adds) into the cluster leader's receive buffer; larger ones are gathered
   // from every CTA's stage buffers (remote atomics serialise at the leader)
   static constexpr bool kPush = PUSH;
   static constexpr int kPushMaxM = 8;
   static_assert(!PUSH || T == 16, "push reduction is for the 16-token tile");
-  static constexpr int kOffRed = kOffSwS + 4 * kTileN;
+  static constexpr int kOffRed = (kOffSx + 4 * T + 15) & ~15;
   static constexpr int kRedBytes = kPush ? T * kTileN * 4 : 0;
   // fused: the cluster-wide per-token absmax (fp32 bit patterns), then this
   // CTA's partial; the quantizing warps hold at most kFusedV float4 each
@@ -269,7 +267,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* ep_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 12);
   float* sx_s = reinterpret_cast<float*>(smem + C::kOffSx);
-  float* sw_s = reinterpret_cast<float*>(smem + C::kOffSwS);
 
   // tile coordinates: the splits of a tile are consecutive blocks (one
   // cluster), then channel blocks, then token blocks (then groups)
@@ -752,9 +749,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
       } else {
         for (int i = et; i < T; i += nthr) sx_s[i] = i < t_valid ? p.s_x[row_base + i] : 0.0f;
       }
-      // this thread's channel scale (loaded before the main loop), staged
-      // for the split-K reduction, which stores other threads' channels
-      if (dg == 0) sw_s[r] = swn;
     }
     warp_wait(bar_acc, 0, abort_flag, lim);
     tc_fence_after();
@@ -886,7 +880,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
 
   if (p.splits > 1 && !push) {
     // ---------------------- split-K by gathering partials over the cluster
-    cluster_sync_all();  // every partial (and every split's ep_flag) is written
+    cluster_sync_all();  // every partial (and every split's ep_flag) is in shared memory
     // a split that aborted wrote no partial: store nothing unless every
     // split of the cluster completed (one remote read per split and warp)
     bool all_ok = false;
@@ -917,38 +911,11 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
       const bool vec_out = (p.N % 4) == 0 &&
                            (p.Y ? (reinterpret_cast<uintptr_t>(p.Y) & 7) == 0
                                 : (reinterpret_cast<uintptr_t>(p.acc) & 15) == 0);
-      // epilogue of one group of 4 channels (element e of the partial tile)
-      auto store4 = [&](int e, const int4& sum) {
-        const int t = e / kTileN, r2 = e % kTileN;
-        const int n2 = n_tile * kTileN + r2;
-        // (channels past N have scale 0 in the staged copy)
-        const float4 sw4 = p.Y ? *reinterpret_cast<const float4*>(sw_s + r2)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-        const int32_t av[4] = {sum.x, sum.y, sum.z, sum.w};
-        const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
-        const size_t o = (size_t)(row_base + t) * p.N + n2;
-        if (vec_out && n2 + 4 <= p.N) {
-          // the group's 4 channels are contiguous in the output row
-          if (p.Y) {
-            const float sx = sx_s[t];
-            uint2 w;
-            w.x = pack_bf16x2((float)av[0] * (sx * swv[0]), (float)av[1] * (sx * swv[1]));
-            w.y = pack_bf16x2((float)av[2] * (sx * swv[2]), (float)av[3] * (sx * swv[3]));
-            *reinterpret_cast<uint2*>(p.Y + o) = w;
-          } else {
-            *reinterpret_cast<int4*>(p.acc + o) = sum;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (n2 + i < p.N) store_out(p, row_base + t, n2 + i, av[i], sx_s[t], swv[i]);
-        }
-      };
       constexpr int kBatch = 2;  // groups in flight per thread and round
       for (int eb = e0 + 4 * et; eb < e1; eb += 4 * nthr * kBatch) {
         // issue every remote load of the round (all splits) before using
-        // any of them: the loads are in flight together, not one round
-        // trip per split
+        // any of them: the loads are in flight together, not one round trip
+        // per split
         int4 got[kClusterMax][kBatch];
 #pragma unroll
         for (int q = 0; q < kClusterMax; ++q) {
@@ -960,18 +927,56 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
                             : make_int4(0, 0, 0, 0);
           }
         }
+        int4 acc4[kBatch];
 #pragma unroll
         for (int b = 0; b < kBatch; ++b) {
-          int4 acc4 = got[0][b];
+          acc4[b] = got[0][b];
 #pragma unroll
           for (int q = 1; q < kClusterMax; ++q) {
-            acc4.x += got[q][b].x;
-            acc4.y += got[q][b].y;
-            acc4.z += got[q][b].z;
-            acc4.w += got[q][b].w;
+            acc4[b].x += got[q][b].x;
+            acc4[b].y += got[q][b].y;
+            acc4[b].z += got[q][b].z;
+            acc4[b].w += got[q][b].w;
           }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
           const int e = eb + 4 * nthr * b;
-          if (e < e1) store4(e, acc4);
+          if (e >= e1) continue;
+          const int t = e / kTileN, r2 = e % kTileN;
+          const int n2 = n_tile * kTileN + r2;
+          // packed s_w is padded to whole channel blocks, so the 4-wide load
+          // is in bounds; the W8 scales are exactly N long
+          float4 sw4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (p.Y) {
+            if (!W8) {
+              sw4 = __ldg(reinterpret_cast<const float4*>(w_scale + n2));
+            } else {
+              sw4.x = __ldg(w_scale + n2);
+              if (n2 + 1 < p.N) sw4.y = __ldg(w_scale + n2 + 1);
+              if (n2 + 2 < p.N) sw4.z = __ldg(w_scale + n2 + 2);
+              if (n2 + 3 < p.N) sw4.w = __ldg(w_scale + n2 + 3);
+            }
+          }
+          const int32_t av[4] = {acc4[b].x, acc4[b].y, acc4[b].z, acc4[b].w};
+          const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
+          const size_t o = (size_t)(row_base + t) * p.N + n2;
+          if (vec_out && n2 + 4 <= p.N) {
+            // the group's 4 channels are contiguous in the output row
+            if (p.Y) {
+              const float sx = sx_s[t];
+              uint2 w;
+              w.x = pack_bf16x2((float)av[0] * (sx * swv[0]), (float)av[1] * (sx * swv[1]));
+              w.y = pack_bf16x2((float)av[2] * (sx * swv[2]), (float)av[3] * (sx * swv[3]));
+              *reinterpret_cast<uint2*>(p.Y + o) = w;
+            } else {
+              *reinterpret_cast<int4*>(p.acc + o) = acc4[b];
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (n2 + i < p.N) store_out(p, row_base + t, n2 + i, av[i], sx_s[t], swv[i]);
+          }
         }
       }
     }
