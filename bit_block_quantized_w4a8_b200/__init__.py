@@ -46,7 +46,7 @@ W4A8_FLAG_TENSOR_CORE = 2  # the tcgen05 kernel even where the decode form appli
 # kernel variants of the ablation study (W4A8_VARIANT_* in include/w4a8.h)
 VARIANTS = {"default": 0, "baseline": 1, "naive_dequant": 2, "serial": 3, "one_group": 4,
             "group_issues_mma": 5, "cta_pair": 6, "tensor_core": 7, "dp4a": 8,
-            "warp_mma": 9}
+            "warp_mma": 9, "persistent": 10}
 
 # kernels behind w4a8_gemm (W4A8_KERNEL_* in include/w4a8.h)
 KERNEL_TENSOR_CORE = 0

@@ -201,6 +201,13 @@ __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+// Waits until every committed bulk store of this thread has read its
+// source in shared memory (the buffer may then be reused; the writes to
+// global memory may still be in flight).
+__device__ __forceinline__ void bulk_wait_group_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Waits until every committed bulk store of this thread has completed
 // (its writes performed), not only read its source.
 __device__ __forceinline__ void bulk_wait_group_all() {

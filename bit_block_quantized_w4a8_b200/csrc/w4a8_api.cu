@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "gemm.cuh"
+#include "gemm_pp.cuh"
 #include "gemv.cuh"
 #include "layout.cuh"
 #include "ptx.cuh"
@@ -354,6 +355,61 @@ bool use_pair(const Schedule& s, const GemmParams& p, bool grouped) {
          p.M >= 256;
 }
 
+// ------------------------------------------------- persistent CTA pairs
+// (gemm_pp.cuh): 192-token tiles, an 8-deep stage ring, 4 weight slots.
+constexpr int kPpTW = 192, kPpSS = 8, kPpAS = 4;
+using PpC = PpCfg<kPpTW, kPpSS, kPpAS>;
+
+// Output tiles of the persistent form for a shape (channel-block pairs x
+// 192-token tiles); 0 when N does not pad to whole pairs.
+long pp_tiles(int M, int N) {
+  const int n_tiles = (N + kTileN - 1) / kTileN;
+  if (n_tiles % 2 != 0) return 0;
+  return (long)(n_tiles / 2) * ((M + kPpTW - 1) / kPpTW);
+}
+
+// The persistent form for a dense call: bf16 output through a TMA store
+// (N a multiple of 8, Y 16-byte aligned), or INT32 output.  Returns
+// cudaErrorNotSupported (nothing launched) when the output does not qualify.
+cudaError_t launch_pp(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
+                      int K, uint16_t* Y, int32_t* acc, cudaStream_t st, bool pdl, int sms) {
+  if (Y && (N % 8 != 0 || !aligned(Y, 16))) return cudaErrorNotSupported;
+  const long tiles = pp_tiles(M, N);
+  if (tiles <= 0) return cudaErrorNotSupported;
+  const int n_pad = round_up(N, kTileN);
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  PpParams p;
+  p.tiles = base + tiles_offset_bytes(n_pad);
+  p.s_w = reinterpret_cast<const float*>(base + sw_offset_bytes());
+  p.s_x = s_x;
+  p.acc = Y ? nullptr : acc;
+  p.hdr = reinterpret_cast<const PackedHeader*>(base);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.kt_total = K / kTileK;
+  p.n_pairs = n_pad / kTileN / 2;
+  p.m_tiles = (M + kPpTW - 1) / kPpTW;
+  p.m_band = p.m_tiles < kRasterBand ? p.m_tiles : kRasterBand;
+  p.wait_limit_ns = wait_budget();
+  CUtensorMap mx, my;
+  if (!make_act_map(&mx, Xq, M, K, kPpTW / 2)) return cudaErrorInvalidValue;
+  my = mx;
+  if (Y && !make_y_map(&my, Y, M, N, kPpTW)) return cudaErrorInvalidValue;
+  auto k = w4a8_gemm_pp_kernel<kPpTW, kPpSS, kPpAS>;
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PpC::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_relaxed);
+  }
+  const long pairs = tiles < sms / 2 ? tiles : sms / 2;
+  return launch_k(k, dim3((unsigned)(2 * pairs)), dim3(PpC::kThreads), PpC::kSmemBytes, st, pdl,
+                  2, mx, my, p);
+}
+
 // Pair launch: the activation box is the CTA's half of the token tile.
 cudaError_t launch_pair(const int8_t* Xq, int M, int K, Maps& m, GemmParams& p, int ctas,
                         cudaStream_t st, bool pdl) {
@@ -587,7 +643,7 @@ struct Groups {
 // at most M rows each).
 // Kernel paths of a dense call: the library's choice, or one forced (the
 // tensor-core kernel, or the CUDA-core decode form).
-enum class Path { kAuto, kTensor, kWarpMma, kDp4a };
+enum class Path { kAuto, kTensor, kWarpMma, kDp4a, kPersist };
 
 int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, int N,
                 int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream,
@@ -598,6 +654,15 @@ int gemm_common(const int8_t* Xq, const float* s_x, const void* packed, int M, i
   if (flags & W4A8_FLAG_TENSOR_CORE) path = Path::kTensor;
   if (g.groups == 0 && path == Path::kDp4a)
     return gemm_gemv(Xq, nullptr, s_x, packed, M, N, K, Y, acc, pdl, stream, false);
+  if (g.groups == 0 && path == Path::kPersist) {  // forced (tests, ablation): any M
+    const int d = current_device();
+    if (d < 0) return W4A8_ERR_CUDA;
+    const cudaError_t e =
+        launch_pp(Xq, s_x, packed, M, N, K, Y, acc, as_stream(stream), pdl, num_sms(d));
+    return e == cudaSuccess ? W4A8_OK
+                            : e == cudaErrorNotSupported ? W4A8_ERR_UNSUPPORTED_SHAPE
+                                                         : W4A8_ERR_CUDA;
+  }
   if (g.groups == 0 &&
       (path == Path::kWarpMma || (path == Path::kAuto && prefer_gemv(M, N, K))))
     return gemm_gemv(Xq, nullptr, s_x, packed, M, N, K, Y, acc, pdl, stream, true);
@@ -721,8 +786,11 @@ int gemm_w8_common(const int8_t* Xq, const float* s_x, const int8_t* Wq, const f
 // reduction; the library's schedule).
 int gemm_variant(int variant, const int8_t* Xq, const float* s_x, const void* packed, int M,
                  int N, int K, uint16_t* Y, int32_t* acc, unsigned flags, void* stream) {
-  if (variant < W4A8_VARIANT_DEFAULT || variant > W4A8_VARIANT_WARP_MMA)
+  if (variant < W4A8_VARIANT_DEFAULT || variant > W4A8_VARIANT_PERSISTENT)
     return W4A8_ERR_INVALID_ARG;
+  if (variant == W4A8_VARIANT_PERSISTENT)
+    return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream, Groups(),
+                       Path::kPersist);
   if (variant == W4A8_VARIANT_DEFAULT)
     return gemm_common(Xq, s_x, packed, M, N, K, Y, acc, flags, stream);
   if (variant == W4A8_VARIANT_TENSOR_CORE)

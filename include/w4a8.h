@@ -259,6 +259,15 @@ int w4a8_gemm_fused_supported(int M, int N, int K);
  *                     K <= 32768 (else W4A8_ERR_UNSUPPORTED_SHAPE)
  *   DP4A              the decode form with CUDA-core 4-way dot products
  *                     (dp4a) instead of warp MMAs; same limits
+ *   PERSISTENT        the persistent CTA-pair form for any M: one CTA pair
+ *                     per two SMs walks 256-channel x 192-token output
+ *                     tiles; two accumulators in tensor memory, so a tile's
+ *                     epilogue (dedicated warps, one TMA store per tile)
+ *                     overlaps the next tile's main loop.  Needs an even
+ *                     number of 128-channel blocks and, for bf16 output, N a
+ *                     multiple of 8 and Y 16-byte aligned (else
+ *                     W4A8_ERR_UNSUPPORTED_SHAPE).  An ablation: measured
+ *                     no faster than CTA_PAIR, so the default never takes it.
  * DEFAULT is the library's own choice (w4a8_gemm_ex / w4a8_gemm_i32).
  * Exactly one of Y (bf16, with s_x) or acc (INT32) is non-NULL.  Other
  * arguments as for w4a8_gemm_ex.
@@ -273,6 +282,7 @@ int w4a8_gemm_fused_supported(int M, int N, int K);
 #define W4A8_VARIANT_TENSOR_CORE 7
 #define W4A8_VARIANT_DP4A 8
 #define W4A8_VARIANT_WARP_MMA 9
+#define W4A8_VARIANT_PERSISTENT 10
 
 int w4a8_gemm_variant(int variant, const int8_t* Xq, const float* s_x,
                       const void* packed, int M, int N, int K, uint16_t* Y,

@@ -8,7 +8,8 @@ still usable: the same call is bit-exact against the oracle.
 
 Every form of the launch is covered once: one CTA per tile, split-K with the
 gather and the push reductions (thread-block clusters), the CTA pair, and
-the warp-MMA decode form with one split and with split-K."""
+the warp-MMA decode form with one split and with split-K, and the persistent
+CTA-pair form."""
 import numpy as np
 import pytest
 import torch
@@ -39,6 +40,7 @@ CASES = [
     (300, 256, 512, "cta_pair", "CTA pairs (tcgen05 cta_group::2)"),
     (2, 256, 512, "warp_mma", "decode form, one split"),
     (2, 256, 8192, "warp_mma", "decode form, split-K 2"),
+    (1000, 512, 1024, "persistent", "persistent CTA pairs, several tiles per pair"),
 ]
 
 

@@ -59,7 +59,7 @@ def test_variant_parity(variant, M, N, K, kind):
 def test_variant_rejections():
     L = w4.lib()
     st = torch.cuda.current_stream().cuda_stream
-    assert L.w4a8_gemm_variant(10, None, None, None, 0, 128, 256, None, None, 0, st) == w4.ERR_INVALID_ARG
+    assert L.w4a8_gemm_variant(11, None, None, None, 0, 128, 256, None, None, 0, st) == w4.ERR_INVALID_ARG
     x = torch.zeros(4, dtype=torch.int32, device="cuda")
     assert L.w4a8_gemm_variant(1, None, None, None, 1, 128, 256, x.data_ptr(), x.data_ptr(), 0, st) == w4.ERR_INVALID_ARG
 
@@ -111,3 +111,66 @@ def test_cta_pair_repeated_runs_are_identical():
         torch.cuda.synchronize()
         assert np.array_equal(acc.cpu().numpy(), acc_ref)
     assert w4.w4a8_get_status() == 0
+
+
+PERSISTENT_CASES = [
+    # (M, N, K, group, kind)
+    (300, 256, 512, 64, "normal"),     # one pair, two tiles (192 + 108 tokens)
+    (1000, 512, 2048, 64, "heavy"),    # 6 token tiles x 2 pairs, last tile 40 rows
+    (4100, 1024, 1024, 64, "ties"),    # 22 token tiles x 4 pairs: some pairs take two rounds
+    (16, 256, 256, 64, "rowzero"),     # a single small tile
+    (500, 200, 384, 128, "normal"),    # ragged N (padded to one pair), group 128
+    (192, 256, 128, 64, "normal"),     # exactly one tile, one k tile
+]
+
+
+@pytest.mark.parametrize("M,N,K,group,kind", PERSISTENT_CASES)
+def test_persistent_pair_parity(M, N, K, group, kind):
+    """The persistent CTA-pair form (double-buffered accumulators, epilogue
+    overlapped with the next tile): INT32 bit-exact, bf16 within 1 ulp of the
+    oracle and bit-identical to the non-persistent kernels."""
+    X = wl.random_matrix(M, K, 300 + M, std=1.0, kind=kind)
+    W = wl.random_matrix(N, K, 301 + N + K, std=0.02)
+    wq = oracle.quantize_weights(W.numpy(), group=group)
+    Xq_ref, sx_ref = oracle.quantize_act(X.numpy())
+    acc_ref, y_ref = oracle.w4a8_gemm(Xq_ref, sx_ref, wq, group=group)
+    pk = w4.w4a8_quantize_weights(W.cuda(), group=group)
+    Xq, sx = w4.w4a8_quantize_act(X.cuda())
+    acc = w4.w4a8_gemm_variant("persistent", Xq, None, pk, i32=True)
+    Y = w4.w4a8_gemm_variant("persistent", Xq, sx, pk, flags=w4.W4A8_FLAG_PDL)
+    Yb = w4.w4a8_gemm_variant("baseline", Xq, sx, pk)
+    torch.cuda.synchronize()
+    assert w4.w4a8_get_status() == 0
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_bf16_within_1ulp(bf16_bits(Y), y_ref, "persistent M=%d N=%d K=%d" % (M, N, K))
+    assert torch.equal(Y.view(torch.int16), Yb.view(torch.int16))
+
+
+def test_persistent_pair_repeated_runs_match_default():
+    """Many tiles per pair (phases carried across tiles), run repeatedly in a
+    PDL chain: the same bits every time, and the same bits as the default
+    call (the per-tile CTA-pair kernel)."""
+    M, N, K = 3000, 2048, 1024
+    X = wl.random_matrix(M, K, 17, std=1.0)
+    W = wl.random_matrix(N, K, 18, std=0.02)
+    pk = w4.w4a8_quantize_weights(W.cuda())
+    Xq, sx = w4.w4a8_quantize_act(X.cuda())
+    ref = w4.w4a8_gemm_variant("baseline", Xq, sx, pk)
+    torch.cuda.synchronize()
+    for _ in range(10):
+        outs = [w4.w4a8_gemm_variant("persistent", Xq, sx, pk, flags=w4.W4A8_FLAG_PDL)
+                for _ in range(3)]
+        torch.cuda.synchronize()
+        for Y in outs:
+            assert torch.equal(Y.view(torch.int16), ref.view(torch.int16))
+    assert w4.w4a8_get_status() == 0
+    Yd = w4.w4a8_gemm(Xq, sx, pk)
+    torch.cuda.synchronize()
+    assert torch.equal(Yd.view(torch.int16), ref.view(torch.int16))
+
+
+def test_persistent_pair_refusals():
+    pk, Xq, sx, _, _ = _case(256, 384, 256, "normal")   # 3 channel blocks: no pairs
+    with pytest.raises(w4.W4A8Error) as e:
+        w4.w4a8_gemm_variant("persistent", Xq, None, pk, i32=True)
+    assert e.value.code == w4.ERR_UNSUPPORTED_SHAPE
