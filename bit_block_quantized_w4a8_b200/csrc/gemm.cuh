@@ -722,6 +722,18 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         tmem_wait_ld();
       }
     };
+    // groups j and j + DQG (when `two`) with one wait: two loads in flight
+    // (the wide tiles' epilogues read up to 8 groups per thread)
+    auto ld_acc2 = [&](int j, bool two, uint32_t (&v)[16], uint32_t (&w)[16]) {
+      if constexpr (kAcc > 1) {
+        ld_acc(j, v);
+        if (two) ld_acc(j + DQG, w);
+      } else {
+        tmem_ld_x16(lane_base + 16 * j, v);
+        if (two) tmem_ld_x16(lane_base + 16 * (j + DQG), w);
+        tmem_wait_ld();
+      }
+    };
     // loads needed only by the epilogue, issued before the main loop so
     // their latency is hidden
     const float swn = (p.Y && n < p.N) ? __ldg(w_scale + n) : 0.0f;  // no scales for INT32 output
@@ -830,20 +842,27 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         // 16-column groups holding valid tokens are read from TMEM, here and
         // below: a 256-token tile at M = 128 carries 128)
         const uint32_t ystage = sbase;
-        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
-          uint32_t v[16];
-          ld_acc(j, v);
-          // two tokens per conversion instruction (the staging is bound by
-          // its per-value work: 2-3% faster prefill than one at a time)
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += 2 * DQG) {
+          const bool two = j + DQG < T / 16 && 16 * (j + DQG) < t_valid;  // warp-uniform
+          uint32_t vv[2][16];
+          ld_acc2(j, two, vv[0], vv[1]);
 #pragma unroll
-          for (int t = 0; t < 16; t += 2) {
-            const int tt = 16 * j + t;
-            const __nv_bfloat162 h =
-                __floats2bfloat162_rn((float)(int32_t)v[t] * (sx_s[tt] * swn),
-                                      (float)(int32_t)v[t + 1] * (sx_s[tt + 1] * swn));
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(&h);
-            sts16(ystage + (uint32_t)(tt * kTileN + r) * 2u, (unsigned short)(w & 0xFFFFu));
-            sts16(ystage + (uint32_t)((tt + 1) * kTileN + r) * 2u, (unsigned short)(w >> 16));
+          for (int hh = 0; hh < 2; ++hh) {
+            if (hh == 1 && !two) break;
+            const int jj = j + hh * DQG;
+            // two tokens per conversion instruction (the staging is bound by
+            // its per-value work: 2-3% faster prefill than one at a time)
+#pragma unroll
+            for (int t = 0; t < 16; t += 2) {
+              const int tt = 16 * jj + t;
+              const __nv_bfloat162 h =
+                  __floats2bfloat162_rn((float)(int32_t)vv[hh][t] * (sx_s[tt] * swn),
+                                        (float)(int32_t)vv[hh][t + 1] * (sx_s[tt + 1] * swn));
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(&h);
+              sts16(ystage + (uint32_t)(tt * kTileN + r) * 2u, (unsigned short)(w & 0xFFFFu));
+              sts16(ystage + (uint32_t)((tt + 1) * kTileN + r) * 2u,
+                    (unsigned short)(w >> 16));
+            }
           }
         }
         fence_proxy_async_smem();  // the stores above, seen by the TMA engine
@@ -855,14 +874,20 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         }
         __syncwarp();
       } else if (p.splits == 1) {
-        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
-          uint32_t v[16];
-          ld_acc(j, v);
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += 2 * DQG) {
+          const bool two = j + DQG < T / 16 && 16 * (j + DQG) < t_valid;  // warp-uniform
+          uint32_t vv[2][16];
+          ld_acc2(j, two, vv[0], vv[1]);
           if (n < p.N) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-              const int tt = 16 * j + t;
-              if (tt < t_valid) store_out(p, row_base + tt, n, (int32_t)v[t], sx_s[tt], swn);
+            for (int hh = 0; hh < 2; ++hh) {
+              if (hh == 1 && !two) break;
+#pragma unroll
+              for (int t = 0; t < 16; ++t) {
+                const int tt = 16 * (j + hh * DQG) + t;
+                if (tt < t_valid)
+                  store_out(p, row_base + tt, n, (int32_t)vv[hh][t], sx_s[tt], swn);
+              }
             }
           }
         }
@@ -871,11 +896,17 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         // (the pipeline buffers are free: every copy landed and every MMA
         // that read them completed)
         int32_t* part = reinterpret_cast<int32_t*>(smem);
-        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
-          uint32_t v[16];
-          ld_acc(j, v);
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += 2 * DQG) {
+          const bool two = j + DQG < T / 16 && 16 * (j + DQG) < t_valid;  // warp-uniform
+          uint32_t vv[2][16];
+          ld_acc2(j, two, vv[0], vv[1]);
 #pragma unroll
-          for (int t = 0; t < 16; ++t) part[(16 * j + t) * kTileN + r] = (int32_t)v[t];
+          for (int hh = 0; hh < 2; ++hh) {
+            if (hh == 1 && !two) break;
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              part[(16 * (j + hh * DQG) + t) * kTileN + r] = (int32_t)vv[hh][t];
+          }
         }
       }
     }
