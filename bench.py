@@ -527,7 +527,8 @@ def run_cuda(args):
         traffic = prof.get("sweep_mean_dram_bytes_per_launch")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": traffic,
-                "kernel": "w4a8_gemm_kernel", "peak_source": peaks["source"],
+                "kernel": "w4a8_gemv_mma_kernel (M <= 16) + w4a8_gemm_kernel (M >= 32)",
+                "peak_source": peaks["source"],
                 "frac_of_spec": achieved / SPEC_HBM_GBS, "spec_gbs": SPEC_HBM_GBS,
                 "note": "algorithmic bytes of the nine sweep launches / their summed average "
                         "launch durations"}
