@@ -244,6 +244,13 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
   const float4* row = reinterpret_cast<const float4*>(X + (size_t)m * K);
   const int n4 = K / 4;
   if (threadIdx.x == 0) pdl_launch_dependents();
+  // The row's lines are requested into L2 before the wait on the preceding
+  // kernel.  A prefetch returns nothing to the thread, so nothing is read
+  // early: if that kernel writes X, its stores land in L2 (the device's point
+  // of coherence) and the loads after the wait read them; if X is older
+  // data, its DRAM latency overlaps the preceding kernel.
+  for (int off = threadIdx.x * 32; off < K; off += kActThreads * 32)
+    prefetch_l2(X + (size_t)m * K + off);
   pdl_wait();  // X may be produced by the preceding kernel
   float4 v[kActRegs];
   float amax = 0.0f;
