@@ -119,6 +119,12 @@ struct GemmCfg {
   // weight stage: one packed LQQ tile, or a 128 x 128 INT8 tile (W8)
   static constexpr int kWBytes = W8 ? kTileN * kTileK : kTileBytes;
   static constexpr int kThreads = (2 + 4 * DQG) * 32;
+  static constexpr int kA0 = T < 32 ? 32 : T;             // first A column
+  static constexpr int kColsUsed = W8 ? kA0 : kA0 + 32 * AS;
+  // a pair allocates all 512 columns, so both CTAs get column address 0
+  static constexpr int kTmemCols = PAIR ? 512 : kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
+                                   : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
+  static_assert(kColsUsed <= 512, "TMEM columns");
   // shared memory: x tiles | w tiles | barriers | misc | s_x cache
   static constexpr int kOffW = SS * kXBytes;
   static constexpr int kOffBar = kOffW + SS * kWBytes;
@@ -221,26 +227,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-// Tensor-memory columns a CTA allocates (a power of two, at least 32).
-__host__ __device__ constexpr int tmem_alloc_cols(int used) {
-  return used <= 32 ? 32 : used <= 64 ? 64 : used <= 128 ? 128 : used <= 256 ? 256 : 512;
-}
-
-// Independent accumulators for narrow token tiles.  Consecutive MMAs into one
-// accumulator form a dependency chain; for a tile of at most 64 tokens each
-// MMA is short and the chain's latency, not the tensor core, sets the pace of
-// a k tile (4 MMAs: measured about 0.42 us per k tile at 16 tokens).  The
-// k-steps of a tile are dealt round-robin over n accumulators (summed in the
-// epilogue), as many as fit in tensor memory with MINB CTAs per SM.
-__host__ __device__ constexpr int tmem_accumulators(int T, int a_cols, int minb, bool pair) {
-  if (pair || T > 64) return 1;
-  for (int n = 4; n > 1; n /= 2) {
-    const int a0 = n * T < 32 ? 32 : n * T;
-    if (tmem_alloc_cols(a0 + a_cols) * minb <= 512) return n;
-  }
-  return 1;
-}
-
 template <int T, int SS, int AS, int DQG, int MINB, bool PUSH, bool W8, int V, bool PAIR,
           bool RTN, bool FUSED>
 __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>::kThreads, MINB)
@@ -252,13 +238,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
   // else the compile-time T (which keeps the full-tile code as tight as it
   // was; a runtime width measured up to 20% slower on full tiles)
   const int TN = RTN ? p.tn : T;
-  // tensor memory: kAcc accumulators of T columns (from column 0), then the
-  // AS dequantized weight slots of 32 columns; a pair allocates all 512
-  // columns, so both CTAs get column address 0
-  constexpr int kAcc = tmem_accumulators(T, W8 ? 0 : 32 * AS, MINB, PAIR);
-  constexpr int kA0 = kAcc * T < 32 ? 32 : kAcc * T;  // first weight-slot column
-  constexpr int kTmemCols = PAIR ? 512 : tmem_alloc_cols(kA0 + (W8 ? 0 : 32 * AS));
-  static_assert(kA0 + (W8 ? 0 : 32 * AS) <= 512 && (PAIR || kTmemCols * MINB <= 512),
+  static_assert(PAIR || C::kTmemCols * MINB <= 512,
                 "tensor-memory columns of the CTAs resident on one SM");
   static_assert(V != kVarGroupIssuesMma || (DQG == 1 && !W8),
                 "the issuing warpgroup must see every k tile");
@@ -391,7 +371,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
       mbar_init(bar_acc, 1);
       mbar_init(bar_done, 4 * DQG);
       mbar_init(bar_red, 1);
-      *abort_flag = 0;
+      *abort_flag = lim == 0 ? 1 : 0;  // a wait budget of 0: abort before any wait
+      if (lim == 0) record_status(kDevTimeout);
       fence_barrier_init();
       // push reduction: the leader's receive barrier completes when every
       // other split's partial (t_valid x 128 INT32 adds) has landed
@@ -410,10 +391,10 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
     __syncwarp();
   } else if (warp == 1) {
     if (PAIR) {
-      tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+      tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
       tmem_relinquish_pair();
     } else {
-      tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+      tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
       tmem_relinquish();
     }
   }
@@ -625,7 +606,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         tc_fence_after();
         if (leader) {
           const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
-          const uint32_t a_tmem = tmem + kA0 + 32 * a;
+          const uint32_t a_tmem = tmem + C::kA0 + 32 * a;
 #pragma unroll
           for (int kk = 0; kk < kTileK / 32; ++kk)
             mma_i8_ts_pair(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc,
@@ -644,56 +625,35 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
     if (FUSED) fused_quant();
     const bool leader = elect_one();
     const uint32_t idesc = idesc_i8(128, TN);
-    // The weights reach the MMA through the dequantized slot (dq), except in
-    // the W8A8 form, which reads the stage's INT8 weight tile directly.
-    // Each round waits for tile `it`, then takes along up to kMmaBatch - 1
-    // further tiles whose operands are ready already (a non-blocking test):
-    // the loop's waits, not the tensor core, set the pace of narrow tiles
-    // (about 0.4 us per k tile with one tile per round at 16 tokens), and
-    // a warp that falls behind catches up in larger rounds.
-    constexpr int kMmaBatch = 4;
-    auto ready = [&](int i) {  // operands of tile i landed (non-blocking)
-      const int s2 = i % SS;
-      const bool w = W8 ? mbar_test_wait(bar_full + 8 * s2, (i / SS) & 1)
-                        : mbar_test_wait(bar_dq + 8 * (i % AS), (i / AS) & 1);
-      return w && mbar_test_wait(bar_fullx + 8 * s2, (i / SS) & 1);
-    };
-    for (int it = 0; it < nk;) {
+    for (int it = 0; it < nk; ++it) {
       const int s = it % SS, a = it % AS;
+      // the weights reach the MMA through the dequantized slot (dq), except
+      // in the W8A8 form, which reads the stage's INT8 weight tile directly
       if (!W8 && !warp_wait(bar_dq + 8 * a, (it / AS) & 1, abort_flag, lim)) break;
       if (W8 && !warp_wait(bar_full + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
       if (!warp_wait(bar_fullx + 8 * s, (it / SS) & 1, abort_flag, lim)) break;
-      // (tile it + cnt's barriers cannot be a phase ahead: their next phase
-      // needs this warp's commits for that tile)
-      int cnt = 1;
-      while (cnt < kMmaBatch && it + cnt < nk && __all_sync(0xffffffffu, ready(it + cnt)))
-        ++cnt;
       tc_fence_after();
       if (leader) {
-        for (int u = 0; u < cnt; ++u) {
-          const int i = it + u, s2 = i % SS, a2 = i % AS;
-          const uint64_t bdesc = smem_desc_sw128(sbase + s2 * C::kXBytes);
-          if (W8) {
-            // both operands in shared memory; +32 bytes of k per instruction
-            const uint64_t adesc = smem_desc_sw128(sbase + C::kOffW + s2 * C::kWBytes);
+        const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
+        if (W8) {
+          // both operands in shared memory; +32 bytes of k per instruction
+          const uint64_t adesc = smem_desc_sw128(sbase + C::kOffW + s * C::kWBytes);
 #pragma unroll
-            for (int kk = 0; kk < kTileK / 32; ++kk)
-              mma_i8_ss(tmem + (uint32_t)((kk % kAcc) * T), adesc + (uint64_t)(2 * kk),
-                        bdesc + (uint64_t)(2 * kk), idesc, i != 0 || kk >= kAcc);
-            tc_commit(bar_empty + 8 * s2);
-          } else {
-            const uint32_t a_tmem = tmem + kA0 + 32 * a2;
+          for (int kk = 0; kk < kTileK / 32; ++kk)
+            mma_i8_ss(tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc,
+                      (it | kk) != 0);
+          tc_commit(bar_empty + 8 * s);
+        } else {
+          const uint32_t a_tmem = tmem + C::kA0 + 32 * a;
 #pragma unroll
-            for (int kk = 0; kk < kTileK / 32; ++kk)
-              mma_i8_ts(tmem + (uint32_t)((kk % kAcc) * T), a_tmem + 8 * kk,
-                        bdesc + (uint64_t)(2 * kk), idesc, i != 0 || kk >= kAcc);
-            tc_commit(bar_empty + 8 * s2);
-            tc_commit(bar_afree + 8 * a2);
-          }
+          for (int kk = 0; kk < kTileK / 32; ++kk)
+            mma_i8_ts(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc,
+                      (it | kk) != 0);
+          tc_commit(bar_empty + 8 * s);
+          tc_commit(bar_afree + 8 * a);
         }
       }
       __syncwarp();
-      it += cnt;
     }
     if (leader) tc_commit(bar_acc);  // also on abort: tracks every MMA issued
     __syncwarp();
@@ -704,36 +664,6 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
     const int r = quarter * 32 + lane;     // weight row in the tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int n = n_tile * kTileN + r;
-    // 16 token columns of this thread's row of the result: the sum of the
-    // kAcc accumulators
-    auto ld_acc = [&](int j, uint32_t (&v)[16]) {
-      tmem_ld_x16(lane_base + 16 * j, v);
-      if constexpr (kAcc > 1) {
-        uint32_t w[kAcc - 1][16];
-#pragma unroll
-        for (int d = 1; d < kAcc; ++d)
-          tmem_ld_x16(lane_base + (uint32_t)(d * T) + 16 * j, w[d - 1]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int d = 1; d < kAcc; ++d)
-#pragma unroll
-          for (int t = 0; t < 16; ++t) v[t] += w[d - 1][t];
-      } else {
-        tmem_wait_ld();
-      }
-    };
-    // groups j and j + DQG (when `two`) with one wait: two loads in flight
-    // (the wide tiles' epilogues read up to 8 groups per thread)
-    auto ld_acc2 = [&](int j, bool two, uint32_t (&v)[16], uint32_t (&w)[16]) {
-      if constexpr (kAcc > 1) {
-        ld_acc(j, v);
-        if (two) ld_acc(j + DQG, w);
-      } else {
-        tmem_ld_x16(lane_base + 16 * j, v);
-        if (two) tmem_ld_x16(lane_base + 16 * (j + DQG), w);
-        tmem_wait_ld();
-      }
-    };
     // loads needed only by the epilogue, issued before the main loop so
     // their latency is hidden
     const float swn = (p.Y && n < p.N) ? __ldg(w_scale + n) : 0.0f;  // no scales for INT32 output
@@ -774,7 +704,7 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
           dequant_chunk(v[c], sc, a4, *reinterpret_cast<uint32_t(*)[8]>(out + 8 * c));
         }
       }
-      tmem_st_x32(lane_base + kA0 + 32 * a, out);
+      tmem_st_x32(lane_base + C::kA0 + 32 * a, out);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -792,11 +722,11 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         tc_fence_after();
         if (elect_one()) {
           const uint64_t bdesc = smem_desc_sw128(sbase + s * C::kXBytes);
-          const uint32_t a_tmem = tmem + kA0 + 32 * a;
+          const uint32_t a_tmem = tmem + C::kA0 + 32 * a;
 #pragma unroll
           for (int kk = 0; kk < kTileK / 32; ++kk)
-            mma_i8_ts(tmem + (uint32_t)((kk % kAcc) * T), a_tmem + 8 * kk,
-                      bdesc + (uint64_t)(2 * kk), idesc_i8(128, TN), it != 0 || kk >= kAcc);
+            mma_i8_ts(tmem, a_tmem + 8 * kk, bdesc + (uint64_t)(2 * kk), idesc_i8(128, TN),
+                      (it | kk) != 0);
           tc_commit(bar_empty + 8 * s);
           tc_commit(bar_afree + 8 * a);
         }
@@ -842,27 +772,21 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         // 16-column groups holding valid tokens are read from TMEM, here and
         // below: a 256-token tile at M = 128 carries 128)
         const uint32_t ystage = sbase;
-        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += 2 * DQG) {
-          const bool two = j + DQG < T / 16 && 16 * (j + DQG) < t_valid;  // warp-uniform
-          uint32_t vv[2][16];
-          ld_acc2(j, two, vv[0], vv[1]);
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
+          uint32_t v[16];
+          tmem_ld_x16(lane_base + 16 * j, v);
+          tmem_wait_ld();
+          // two tokens per conversion instruction (the staging is bound by
+          // its per-value work: 2-3% faster prefill than one at a time)
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            if (hh == 1 && !two) break;
-            const int jj = j + hh * DQG;
-            // two tokens per conversion instruction (the staging is bound by
-            // its per-value work: 2-3% faster prefill than one at a time)
-#pragma unroll
-            for (int t = 0; t < 16; t += 2) {
-              const int tt = 16 * jj + t;
-              const __nv_bfloat162 h =
-                  __floats2bfloat162_rn((float)(int32_t)vv[hh][t] * (sx_s[tt] * swn),
-                                        (float)(int32_t)vv[hh][t + 1] * (sx_s[tt + 1] * swn));
-              const uint32_t w = *reinterpret_cast<const uint32_t*>(&h);
-              sts16(ystage + (uint32_t)(tt * kTileN + r) * 2u, (unsigned short)(w & 0xFFFFu));
-              sts16(ystage + (uint32_t)((tt + 1) * kTileN + r) * 2u,
-                    (unsigned short)(w >> 16));
-            }
+          for (int t = 0; t < 16; t += 2) {
+            const int tt = 16 * j + t;
+            const __nv_bfloat162 h =
+                __floats2bfloat162_rn((float)(int32_t)v[t] * (sx_s[tt] * swn),
+                                      (float)(int32_t)v[t + 1] * (sx_s[tt + 1] * swn));
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(&h);
+            sts16(ystage + (uint32_t)(tt * kTileN + r) * 2u, (unsigned short)(w & 0xFFFFu));
+            sts16(ystage + (uint32_t)((tt + 1) * kTileN + r) * 2u, (unsigned short)(w >> 16));
           }
         }
         fence_proxy_async_smem();  // the stores above, seen by the TMA engine
@@ -874,20 +798,15 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         }
         __syncwarp();
       } else if (p.splits == 1) {
-        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += 2 * DQG) {
-          const bool two = j + DQG < T / 16 && 16 * (j + DQG) < t_valid;  // warp-uniform
-          uint32_t vv[2][16];
-          ld_acc2(j, two, vv[0], vv[1]);
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
+          uint32_t v[16];
+          tmem_ld_x16(lane_base + 16 * j, v);
+          tmem_wait_ld();
           if (n < p.N) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              if (hh == 1 && !two) break;
-#pragma unroll
-              for (int t = 0; t < 16; ++t) {
-                const int tt = 16 * (j + hh * DQG) + t;
-                if (tt < t_valid)
-                  store_out(p, row_base + tt, n, (int32_t)vv[hh][t], sx_s[tt], swn);
-              }
+            for (int t = 0; t < 16; ++t) {
+              const int tt = 16 * j + t;
+              if (tt < t_valid) store_out(p, row_base + tt, n, (int32_t)v[t], sx_s[tt], swn);
             }
           }
         }
@@ -896,17 +815,12 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
         // (the pipeline buffers are free: every copy landed and every MMA
         // that read them completed)
         int32_t* part = reinterpret_cast<int32_t*>(smem);
-        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += 2 * DQG) {
-          const bool two = j + DQG < T / 16 && 16 * (j + DQG) < t_valid;  // warp-uniform
-          uint32_t vv[2][16];
-          ld_acc2(j, two, vv[0], vv[1]);
+        for (int j = dg; j < T / 16 && 16 * j < t_valid; j += DQG) {
+          uint32_t v[16];
+          tmem_ld_x16(lane_base + 16 * j, v);
+          tmem_wait_ld();
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            if (hh == 1 && !two) break;
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-              part[(16 * (j + hh * DQG) + t) * kTileN + r] = (int32_t)vv[hh][t];
-          }
+          for (int t = 0; t < 16; ++t) part[(16 * j + t) * kTileN + r] = (int32_t)v[t];
         }
       }
     }
@@ -927,7 +841,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
           if (16 * j >= t_valid) break;
           uint32_t v[16];
           if (live) {
-            ld_acc(j, v);
+            tmem_ld_x16(lane_base + 16 * j, v);
+            tmem_wait_ld();
           } else {
 #pragma unroll
             for (int t = 0; t < 16; ++t) v[t] = 0;
@@ -948,7 +863,8 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
           for (int j = dg; j < T / 16; j += DQG) {
             if (16 * j >= t_valid) break;
             uint32_t v[16];
-            ld_acc(j, v);
+            tmem_ld_x16(lane_base + 16 * j, v);
+            tmem_wait_ld();
             if (n < p.N) {
 #pragma unroll
               for (int t = 0; t < 16; ++t) {
@@ -1091,9 +1007,9 @@ __global__ void __launch_bounds__(GemmCfg<T, SS, AS, DQG, PUSH, W8, PAIR, FUSED>
     if (FUSED && p.splits > 1) warp_wait<true>(bar_amax, 0, nullptr, kDrainLimitNs);
     tc_fence_after();
     if (PAIR)
-      tmem_dealloc_pair(tmem, kTmemCols);
+      tmem_dealloc_pair(tmem, C::kTmemCols);
     else
-      tmem_dealloc(tmem, kTmemCols);
+      tmem_dealloc(tmem, C::kTmemCols);
   }
   __syncwarp();
   __syncthreads();

@@ -135,7 +135,8 @@ __global__ void __launch_bounds__(PpCfg<TW, SS, AS>::kThreads, 1)
       }
       mbar_init(bar_fin, 1);
       mbar_init(bar_done, C::kEpiWarps);
-      *abort_flag = 0;
+      *abort_flag = lim == 0 ? 1 : 0;  // a wait budget of 0: abort before any wait
+      if (lim == 0) record_status(kDevTimeout);
       fence_barrier_init();
       pdl_launch_dependents();
     }

@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(kGemvThreads, MINB)
     mbar_init(bar_w, 1);
     mbar_init(bar_x, 1);
     mbar_init(bar_red, 1);
-    *abort_flag = 0;
+    *abort_flag = lim == 0 ? 1 : 0;  // a wait budget of 0: abort before any wait
+    if (lim == 0) record_status(kDevTimeout);
     fence_barrier_init();
     if (p.splits > 1 && leader)
       mbar_arrive_expect_tx(bar_red, (uint32_t)(p.splits - 1) * (uint32_t)(M * R * 4));
@@ -415,7 +416,8 @@ __global__ void __launch_bounds__(kGemvThreads, MINB)
     mbar_init(bar_w, 1);
     mbar_init(bar_x, 1);
     mbar_init(bar_red, 1);
-    *abort_flag = 0;
+    *abort_flag = lim == 0 ? 1 : 0;  // a wait budget of 0: abort before any wait
+    if (lim == 0) record_status(kDevTimeout);
     fence_barrier_init();
     if (p.splits > 1 && leader)
       mbar_arrive_expect_tx(bar_red, (uint32_t)(p.splits - 1) * (uint32_t)(M * R * 4));
