@@ -445,5 +445,6 @@ def w4a8_debug_timeout_probe(limit_ns, stream=None):
 
 def w4a8_debug_set_wait_budget(ns):
     """Test aid: budget of the kernels' main-loop waits for later launches
-    (-1 = the default 2 s; 0 = expire at once, so every launch aborts)."""
+    (-1 = the default 2 s; 0 = every CTA raises its abort flag at set-up,
+    so every launch aborts)."""
     _check(lib().w4a8_debug_set_wait_budget(int(ns)), "w4a8_debug_set_wait_budget")

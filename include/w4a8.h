@@ -382,7 +382,9 @@ int w4a8_debug_timeout_probe(long long limit_ns, void* stream);
  * Test aid for the GEMM's own failure path: the budget, in nanoseconds, of
  * the main-loop waits of every kernel launched afterwards by this process
  * (all entry points, all devices).  -1 restores the default of 2 s; 0 makes
- * every such wait expire at once, so each launch runs its abort path: the
+ * every CTA of each launch raise its abort flag at set-up, before any wait,
+ * so each of those waits that does not find its phase complete gives up at
+ * once and the launch runs its abort path: the
  * status word records W4A8_ERR_TIMEOUT, nothing is stored, and the kernel
  * first waits (always with the full 2 s budget) for the copies, MMAs and
  * remote adds it already started, then frees its tensor memory and returns.

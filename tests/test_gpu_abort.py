@@ -1,6 +1,7 @@
 """The GEMM kernels' own failure path on the GPU, without a fault: with the
-test wait budget set to 0 (w4a8_debug_set_wait_budget) every main-loop wait
-of a launch expires at once, so each CTA runs its abort path -- it records
+test wait budget set to 0 (w4a8_debug_set_wait_budget) every CTA of a launch
+raises its abort flag at set-up, so each main-loop wait that does not find
+its phase complete gives up at once and each CTA runs its abort path -- it records
 W4A8_ERR_TIMEOUT, stores nothing, waits with the full 2 s budget for the
 copies, MMAs and remote adds it already started, frees its tensor memory and
 returns.  The test then restores the budget and checks that the context is
