@@ -1033,7 +1033,7 @@ def run_ablation(args):
               ("llama70b_like", "down", [512]),
               ("prefill", "square8k", [8192])]
     variants = ["default", "baseline", "naive_dequant", "serial", "one_group",
-                "group_issues_mma", "cta_pair"]
+                "group_issues_mma", "cta_pair", "tensor_core", "warp_mma", "dp4a", "persistent"]
     out = {"peaks": peaks, "variants": variants, "cases": []}
     for name, lname, Ms in shapes:
         layer = [L for L in wl.WORKLOADS[name].layers if L.name == lname][0]
@@ -1051,8 +1051,12 @@ def run_ablation(args):
             n_in = 8 if M < 4096 else 2
             t = {}
             for v in variants:
-                if v == "cta_pair" and (M < 256 or (-(-N // 128)) % 2):
-                    continue  # the pair form needs full 256-token tiles, paired channel blocks
+                if v in ("cta_pair", "persistent") and (M < 256 or (-(-N // 128)) % 2):
+                    continue  # the pair forms need full 256-token tiles, paired channel blocks
+                if (v == "warp_mma" and M > 16) or (v == "dp4a" and M > 8):
+                    continue  # the decode form's token limits
+                if v == "tensor_core" and M > 16:
+                    continue  # the default is the tensor-core kernel already
                 def body(v=v):
                     for i in range(n_in):
                         w4.w4a8_gemm_variant(v, Xq, sx, copies[i % ncopy], out=Y, stream=stream,
